@@ -1,0 +1,263 @@
+/*
+ * zha.h: C ABI of the B200 library for Zyphra Hierarchical Attention (ZHA).
+ *
+ * ZHA keeps, beside an unchanged KV cache, a tree of compressed key summaries.
+ * A node summarizes C consecutive nodes of the level below (C consecutive keys at
+ * level 1) and holds, for each of R reference queries q_r, one tangent of the
+ * region's log-sum-exp attention: a key and a bias. A query walks the tree from
+ * the top, opening nodes level by level by top-p mass or top-K, and ordinary
+ * attention then runs over exactly the original keys of the opened level-1
+ * nodes.
+ *
+ * Sources (page, then section):
+ *   [P1] "How does a tree of summaries search a context? How ZHA works"
+ *        (learn.chabulab.com): "How is the tree built?", "What does a node
+ *        summarize?", "How does top-p differ from top-K?", "Run a small tree
+ *        yourself", "Common misunderstandings".
+ *   [P4] "Subquadratic Attention with a Hierarchical Tree-Structured Indexer",
+ *        abstract (tree of recursively compressed key summaries, traversed from
+ *        the top down; sublinear routing plus final attention).
+ *   [P3] "Zyphra AI Introduces ZHA, a Path to True Subquadratic Attention"
+ *        (full-scan indexers score every token).
+ *
+ * Conventions for every call:
+ *   - Pointers named K, V, Q, k_new, v_new, refs, sel, sel_count, out, lse and
+ *     stats are DEVICE pointers (CUDA global memory of the current device), owned
+ *     by the caller. The library never frees them.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream): arguments are checked on the host before anything is
+ *     launched; results are ready when the stream reaches that point.
+ *   - Every call returns ZHA_OK (0) or a negative ZHA_ERR_* code and records a
+ *     message readable with zha_last_error() (per host thread). No call aborts
+ *     the process, and no exception crosses this boundary.
+ *   - Errors the device finds (e.g. a walk opening more chunks than max_sel)
+ *     are recorded in the tree and returned by zha_sync_status().
+ *   - Layouts are row-major. B = batch (sequences), H_kv = KV heads, H_q = query
+ *     heads (a multiple of H_kv; query head h uses KV head h / (H_q / H_kv)),
+ *     d = head dimension, n_q = queries per query head. A "walk" is one query
+ *     vector of one query head; walk w = (b * H_q + h) * n_q + i, so that the
+ *     walks of tree t = b * H_kv + h_kv are the contiguous ids
+ *     t * G .. t * G + G - 1 with G = (H_q / H_kv) * n_q.
+ */
+#ifndef ZHA_H
+#define ZHA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ZHA_MAX_DEPTH 12
+
+typedef enum {
+    ZHA_OK = 0,
+    ZHA_ERR_INVALID = -1,  /* bad argument: NULL pointer, shape, dtype, range */
+    ZHA_ERR_CAPACITY = -2, /* append past capacity; a walk needed more than max_sel */
+    ZHA_ERR_OOM = -3,      /* device allocation failed */
+    ZHA_ERR_CUDA = -4,     /* a CUDA call or launch failed (message has the CUDA error) */
+    ZHA_ERR_INTERNAL = -5, /* a device-side consistency check failed */
+    ZHA_ERR_TIMEOUT = -6   /* reserved for bounded device-side waits */
+} zha_status;
+
+typedef enum { ZHA_F32 = 0, ZHA_BF16 = 1 } zha_dtype;
+typedef enum { ZHA_TOP_P = 0, ZHA_TOP_K = 1 } zha_mode;
+
+/* Shape and parameters of a set of trees (one per sequence and KV head). */
+typedef struct {
+    int batch;          /* B >= 1 */
+    int n_kv_heads;     /* H_kv >= 1 */
+    int d;              /* head dimension: 64, 128 or 256 */
+    int R;              /* reference queries per tree, 1..16 */
+    int chunk;          /* C: children per node, 2..64 */
+    int depth;          /* levels built, 1..ZHA_MAX_DEPTH */
+    int top_width;      /* a walk starts at the lowest level holding at most this
+                           many nodes (the deepest level if none does); >= 1.
+                           [P1] "Run a small tree yourself": the demo's top level
+                           has at most 64 nodes. */
+    long long capacity; /* keys per tree that K and V can hold, >= 1 */
+    float sharpness;    /* beta: scale of every query-key dot product, both in the
+                           summaries and in the final attention (1/sqrt(d) for a
+                           standard attention head) */
+    zha_dtype kv_dtype; /* element type of K, V, k_new, v_new and out */
+} zha_config;
+
+/* Per-walk counters written by zha_search when `stats` is not NULL.
+   [P1] "Try it" / "Run a small tree yourself": the demo counts one comparison
+   per reference query per frontier node, plus one per key read. */
+typedef struct {
+    int start_level;                /* level the walk started at */
+    int frontier[ZHA_MAX_DEPTH + 1];/* nodes scored at each level (index = level) */
+    int opened[ZHA_MAX_DEPTH + 1];  /* nodes opened at each level */
+    long long keys_read;            /* C * opened level-1 nodes + tail keys */
+    long long work;                 /* R * sum(frontier) + keys_read */
+} zha_stats;
+
+/* Opaque handle: the level arrays of B * H_kv trees, plus scratch for searches.
+   Owned by the library; freed by zha_destroy. */
+typedef struct zha_tree zha_tree;
+
+/*
+ * zha_build: build every level of every tree over the first n_keys keys.
+ *   [P1] "How is the tree built?" and "What does a node summarize?": node j of
+ *   level l summarizes nodes C*j .. C*j+C-1 of level l-1 (keys at level 1); for
+ *   each reference r, with child scores s_i = beta*<key_{i,r}, q_r> + bias_{i,r}
+ *   (bias 0 for keys), the node keeps key_r = sum_i softmax(s)_i key_{i,r} and
+ *   bias_r = logsumexp(s) - beta*<key_r, q_r>. Level l has floor(n_{l-1}/C)
+ *   nodes; keys past the last full chunk (the tail) have no node yet.
+ * K, V:  [B][H_kv][capacity][d] of cfg->kv_dtype, the caller's KV cache. The tree
+ *        keeps these pointers: zha_append writes new keys and values into them,
+ *        and zha_build, zha_append and zha_attend read them. Both must stay
+ *        valid until zha_destroy.
+ * refs:  [H_kv][R][d] fp32, the reference queries of each KV head (shared by all
+ *        sequences). Kept by pointer like K and V.
+ * n_keys: 0 .. capacity.
+ * out:   receives the new handle (set to NULL on error).
+ * Node storage is allocated here for `capacity` keys: level l holds
+ * floor(capacity / C^l) nodes of R*d + round_up(R, 4) fp32 each (keys [R][d],
+ * then biases [R], then padding).
+ * Errors: ZHA_ERR_INVALID (NULL pointer, shape out of range, n_keys > capacity),
+ * ZHA_ERR_OOM, ZHA_ERR_CUDA.
+ */
+int zha_build(const zha_config *cfg, void *K, void *V, const float *refs, long long n_keys,
+              void *stream, zha_tree **out);
+
+/*
+ * zha_append: append one key and one value to every tree at position n (the
+ * current key count), then make the nodes whose chunk this fills: the level-1
+ * node if (n+1) % C == 0, its parent if that completes a group of C at level 1,
+ * and so on up to `depth`. [P1] "How is the tree built?": a node is created each
+ * time a chunk fills. The result equals zha_build over the n+1 keys.
+ * k_new, v_new: [B][H_kv][d] of kv_dtype (device).
+ * Errors: ZHA_ERR_INVALID (NULL), ZHA_ERR_CAPACITY (n == capacity), ZHA_ERR_CUDA.
+ */
+int zha_append(zha_tree *tree, const void *k_new, const void *v_new, void *stream);
+
+/*
+ * zha_search: walk every query down its tree ([P1] "Run a small tree yourself",
+ * route; "How does top-p differ from top-K?").
+ *   1. The frontier starts as every node of the start level (see top_width).
+ *   2. Each frontier node scores max_r (beta*<key_r, q> + bias_r) ([P1] "What
+ *      does a node summarize?": a tangent per reference, take the highest).
+ *   3. mass = softmax of the scores over the whole frontier of the walk.
+ *   4. Top-p: open the shortest prefix of the nodes ordered by mass (descending,
+ *      ties by ascending node id) whose mass sums to at least p; p >= 1 opens
+ *      all. Top-K: open the K nodes first in that order (all if fewer).
+ *   5. The next frontier is the children of the opened nodes plus the nodes of
+ *      the level below whose parent does not exist yet (orphans); at level 1 the
+ *      opened nodes are the result.
+ * Q:        [B][H_q][n_q][d] of q_dtype.
+ * sel:      [walks][max_sel] int32: opened level-1 node ids, ascending; entries
+ *           past sel_count are unspecified.
+ * sel_count:[walks] int32. Keys [C*n_1, n) (the tail) are always attended too.
+ * stats:    NULL or [walks] zha_stats.
+ * mode/p/k: ZHA_TOP_P with 0 < p (p >= 1 opens everything), or ZHA_TOP_K with
+ *           k >= 1.
+ * Scratch memory is taken from the tree (grown on first use for this many
+ * walks; see zha_reserve).
+ * Errors: ZHA_ERR_INVALID, ZHA_ERR_OOM, ZHA_ERR_CUDA; a walk that opens more than
+ * max_sel level-1 nodes keeps the first max_sel (ascending) and makes
+ * zha_sync_status return ZHA_ERR_CAPACITY.
+ */
+int zha_search(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q,
+               zha_mode mode, float p, int k, int *sel, int *sel_count, int max_sel,
+               zha_stats *stats, void *stream);
+
+/*
+ * zha_attend: attention of every walk over exactly its chosen keys: the keys of
+ * the level-1 nodes in sel plus the tail keys [C*n_1, n) ([P1] "How is the tree
+ * built?" and "Common misunderstandings": the final attention runs on the
+ * original keys and values). out = sum_i softmax_i(beta*<q, k_i>) v_i,
+ * lse = logsumexp_i(beta*<q, k_i>), both accumulated in fp32.
+ * Q:   [B][H_q][n_q][d] of q_dtype; sel/sel_count as written by zha_search.
+ * out: [B][H_q][n_q][d] of out_dtype (the fp32 result, rounded to nearest even
+ *      for ZHA_BF16); lse: [walks] fp32 (may be NULL).
+ * A walk with no key at all (n == 0) gets out = 0 and lse = -inf.
+ * Errors: ZHA_ERR_INVALID, ZHA_ERR_OOM, ZHA_ERR_CUDA; a sel id out of range makes
+ * zha_sync_status return ZHA_ERR_INTERNAL (the id is skipped).
+ */
+int zha_attend(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q,
+               const int *sel, const int *sel_count, int max_sel, void *out, zha_dtype out_dtype,
+               float *lse, void *stream);
+
+/*
+ * zha_reserve: allocate the search and attend scratch for up to max_walks walks
+ * and selections of up to max_sel chunks now, so that later calls with at most
+ * these sizes allocate nothing (e.g. before capturing them in a CUDA graph).
+ */
+int zha_reserve(zha_tree *tree, long long max_walks, int max_sel);
+
+/*
+ * zha_level: device pointer to the node array of one level (1..depth) of all
+ * trees, laid out [B*H_kv][level_capacity][node_floats] fp32 with node_floats =
+ * R*d + round_up(R, 4) (keys [R][d], biases [R], padding); the live node count
+ * per tree is written to *n_nodes and the per-tree capacity to *level_capacity.
+ * The pointer stays owned by the tree. For inspection and tests.
+ */
+int zha_level(const zha_tree *tree, int level, const float **nodes, long long *n_nodes,
+              long long *level_capacity, int *node_floats);
+
+/* ---------------------------------------------------------------------------
+ * Diagnostics (not on the hot path): kernel timing, launch counts and the size of
+ * the last search's frontiers, used by the benchmark's roofline figures.
+ */
+typedef enum {
+    ZHA_K_BUILD = 0,          /* node summaries (build and append) */
+    ZHA_K_APPEND = 1,         /* key/value write of zha_append */
+    ZHA_K_SEARCH_INIT = 2,    /* walk set-up */
+    ZHA_K_SCORE = 3,          /* frontier scoring, one launch per level */
+    ZHA_K_SELECT = 4,         /* top-p / top-K selection and expansion, one per level */
+    ZHA_K_ATTEND_PLAN = 5,    /* split of each walk's keys into work items */
+    ZHA_K_ATTEND_PARTIAL = 6, /* gathered attention over the chosen keys */
+    ZHA_K_ATTEND_COMBINE = 7, /* log-sum-exp merge of the partial results */
+    ZHA_K_KINDS = 8
+} zha_kernel_kind;
+
+typedef struct {
+    long long launches; /* launches recorded */
+    double ms;          /* summed device time between the CUDA events around them */
+} zha_kernel_time;
+
+/* zha_profile: enable (1) or disable (0) recording a CUDA event pair on the
+ * launching stream around every kernel this tree launches. */
+int zha_profile(zha_tree *tree, int enable);
+
+/* zha_profile_read: waits for `stream`, writes the per-kind totals recorded since
+ * the last read into out[ZHA_K_KINDS] and clears them. */
+int zha_profile_read(zha_tree *tree, zha_kernel_time *out, void *stream);
+
+/* Kernels launched by this library in this process, all trees together. */
+long long zha_kernel_launches(void);
+
+/* Size of the frontiers of the last zha_search on this tree. */
+typedef struct {
+    int start_level;
+    long long union_nodes[ZHA_MAX_DEPTH + 1]; /* sum over trees of |union of the walks' frontiers| per level */
+    long long walk_nodes[ZHA_MAX_DEPTH + 1];  /* sum over walks of |frontier| per level */
+} zha_search_info;
+
+/* zha_last_search_info: waits for `stream` and counts the frontier bits the last
+ * zha_search left in its scratch. Valid until the next search on this tree. */
+int zha_last_search_info(zha_tree *tree, zha_search_info *out, void *stream);
+
+/* Keys currently in every tree (n). */
+long long zha_num_keys(const zha_tree *tree);
+
+/* Waits for the tree's pending work on `stream`, then returns and clears the
+   first device-side error recorded since the last call (ZHA_OK if none). */
+int zha_sync_status(zha_tree *tree, void *stream);
+
+/* Frees the tree's node storage and scratch. NULL is a no-op. Pending work that
+   uses the tree must have finished. */
+void zha_destroy(zha_tree *tree);
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char *zha_last_error(void);
+
+/* Library version string. */
+const char *zha_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ZHA_H */

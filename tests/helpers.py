@@ -1,0 +1,106 @@
+"""Shared helpers of the parity tests: the oracle side of a workload, and the
+element-wise comparisons with the tolerances the method's targets fix.
+
+Tolerances (per element g = GPU, o = oracle):
+  node keys and biases: |g - o| <= rtol * max|o over the row|, rtol = 1e-5 (a row
+      = one reference key of a node, or a node's R biases): 1e-5 relative to the
+      magnitude of the vector the element belongs to. An element near zero is a
+      cancellation of weighted terms of the row's size, so fp32 gives it an
+      absolute error of a few ulps of the row, not of itself;
+  attention outputs (fp32) and lse: |g - o| <= atol * max(1, |o|), atol = 1e-5
+      for an fp32 cache and 3e-3 for a bf16 cache;
+  attention outputs stored as bf16: within one bf16 ulp of the oracle's output
+      rounded to bf16 (rounding alone moves a value by up to 2^-8 relative, more
+      than 3e-3, and values near a rounding boundary may round either way);
+  selected chunk sets: identical, unless the oracle's walk met a near-tie: a
+      relative gap below 1e-5 between the last opened and the first unopened
+      mass, or a running top-p sum within 1e-5 * p of p.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as O
+
+NODE_RTOL = 1e-5
+TIE_TOL = 1e-5
+
+
+def attn_tol(w) -> float:
+    return 1e-5 if w.kv_dtype == "f32" else 3e-3
+
+
+def host64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def oracle_tree(inp, b: int, h: int, n_keys: int | None = None, threads: int = 0, capacity=None):
+    w = inp.w
+    n = w.n_keys if n_keys is None else n_keys
+    K = host64(inp.K[b, h, :n])
+    refs = host64(inp.refs[h])
+    return O.build_tree(K, refs, w.chunk, w.depth, w.beta, store=O.STORE_F32, threads=threads,
+                        capacity=capacity)
+
+
+def gpu_level(tree, l: int, t: int):
+    nodes, n = tree.level(l)
+    return host64(nodes[t, :n]), n
+
+
+def assert_nodes_close(g: np.ndarray, keys: np.ndarray, bias: np.ndarray, R: int, d: int,
+                       rtol: float = NODE_RTOL, what: str = ""):
+    n = keys.shape[0]
+    assert g.shape[0] == n, (what, g.shape, keys.shape)
+    gk = g[:, : R * d].reshape(n, R, d)
+    gb = g[:, R * d: R * d + R]
+    scale_k = np.abs(keys).max(axis=2, keepdims=True)
+    bad_k = np.abs(gk - keys) > rtol * scale_k
+    assert not bad_k.any(), f"{what}: {bad_k.sum()} node key elements off; worst |diff| " \
+                            f"{np.abs(gk - keys).max():.3g}"
+    scale_b = np.abs(bias).max(axis=1, keepdims=True)
+    bad_b = np.abs(gb - bias) > rtol * scale_b
+    assert not bad_b.any(), f"{what}: {bad_b.sum()} biases off; worst |diff| {np.abs(gb - bias).max():.3g}"
+
+
+def near_tie(walk) -> bool:
+    return min(walk.tie_gap, walk.tie_sum) < TIE_TOL
+
+
+def compare_selection(sel: np.ndarray, cnt: np.ndarray, walks: dict):
+    """walks: {walk index: oracle Walk}. Returns the walk ids that differ (each of
+    them must be a near-tie in the oracle)."""
+    differ = []
+    for w, ow in walks.items():
+        g = sel[w, : cnt[w]]
+        if not np.array_equal(g, ow.sel):
+            assert near_tie(ow), (f"walk {w}: GPU and oracle selections differ away from a tie "
+                                  f"(gap {ow.tie_gap:.3g}, sum {ow.tie_sum:.3g}; "
+                                  f"{len(g)} vs {len(ow.sel)} chunks)")
+            differ.append(w)
+    return differ
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    import torch as _t
+
+    return _t.from_numpy(np.asarray(x, dtype=np.float32)).to(_t.bfloat16).to(_t.float64).numpy()
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+def assert_bf16_output_close(out_g: np.ndarray, out_o: np.ndarray, what: str = ""):
+    r = bf16_round(out_o)
+    bad = np.abs(out_g - r) > bf16_ulp(r) * 1.0001
+    assert not bad.any(), f"{what}: {bad.sum()} bf16 outputs more than one ulp from the rounded oracle"
+
+
+def assert_attention_close(out_g: np.ndarray, lse_g: float, out_o: np.ndarray, lse_o: float, atol: float,
+                           what: str = ""):
+    err = np.abs(out_g - out_o) / np.maximum(1.0, np.abs(out_o))
+    assert err.max() <= atol, f"{what}: attention output off by {err.max():.3g} (tol {atol})"
+    assert abs(lse_g - lse_o) <= atol * max(1.0, abs(lse_o)), f"{what}: lse {lse_g} vs {lse_o}"

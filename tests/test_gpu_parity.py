@@ -1,0 +1,334 @@
+"""GPU parity: the CUDA library (through its C ABI) against the oracle, on the same
+seeded inputs, at sizes the oracle finishes in seconds (several tiles, ragged
+tails, orphans, GQA groups, several queries per head).
+
+What is compared, per workload and mode:
+  * every node key and bias of every level of every tree (1e-5 relative);
+  * every walk's selected chunk set (identical except at oracle near-ties, which
+    are counted and printed) and its counters (frontier and opened per level,
+    keys read, comparisons);
+  * the attention over the oracle's own selection (GPU attend fed the oracle's
+    chunk lists), and the end-to-end search + attend where the sets agree;
+  * p = 1 against dense attention.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synthetic as S
+from helpers import (assert_attention_close, assert_bf16_output_close, assert_nodes_close, attn_tol,
+                     compare_selection, gpu_level, host64, oracle_tree)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "demo4k": S.WORKLOADS["demo4k"],
+    "demo4k_iid": S.control(S.WORKLOADS["demo4k"]),
+    "kv64k": S.WORKLOADS["kv64k"],
+    "kv256k_small": S.scaled(S.WORKLOADS["kv256k"], name="kv256k_small", batch=2, n_keys=32768 + 5 * 8 + 3,
+                             depth=5, appends=512),
+    "kv1m_small": S.scaled(S.WORKLOADS["kv1m"], name="kv1m_small", batch=1, n_keys=65536, depth=4),
+}
+
+MODE = {"top_p": O.TOP_P, "top_k": O.TOP_K}
+
+
+def zha():
+    import tree_indexed_sparse_append_b200 as Z
+
+    return Z
+
+
+def walk_index(w, b, hq, i):
+    return (b * w.n_q_heads + hq) * w.queries_per_head + i
+
+
+class Case:
+    def __init__(self, name, w):
+        self.name, self.w = name, w
+        self.inp = S.draw(w, device="cuda")
+        self.tree = zha().Tree(self.inp.K, self.inp.V, self.inp.refs, w.n_keys, w.chunk, w.depth, w.beta,
+                               w.top_width)
+        torch.cuda.synchronize()
+        self.otrees = {(b, h): oracle_tree(self.inp, b, h, threads=8)
+                       for b in range(w.batch) for h in range(w.n_kv_heads)}
+        self.Kh = {k: host64(self.inp.K[k[0], k[1], : w.n_keys]) for k in self.otrees}
+        self.Vh = {k: host64(self.inp.V[k[0], k[1], : w.n_keys]) for k in self.otrees}
+        self.Qh = host64(self.inp.Q)
+
+    def walks(self):
+        w = self.w
+        group = w.n_q_heads // w.n_kv_heads
+        for b in range(w.batch):
+            for hq in range(w.n_q_heads):
+                for i in range(w.queries_per_head):
+                    yield walk_index(w, b, hq, i), (b, hq // group), self.Qh[b, hq, i]
+
+    def oracle_search(self, mode, p, k):
+        return {wi: O.search(self.otrees[key], q, MODE[mode], p, k, self.w.top_width)
+                for wi, key, q in self.walks()}
+
+
+@pytest.fixture(scope="module", params=list(SMALL))
+def case(request):
+    c = Case(request.param, SMALL[request.param])
+    yield c
+    c.tree.close()
+    del c
+    torch.cuda.empty_cache()
+
+
+def test_build_matches_oracle(case):
+    w = case.w
+    for (b, h), ot in case.otrees.items():
+        t = b * w.n_kv_heads + h
+        for l in range(1, w.depth + 1):
+            g, n = gpu_level(case.tree, l, t)
+            assert n == ot.n_nodes[l]
+            keys, bias = ot.level(l)
+            assert_nodes_close(g, keys, bias, w.R, w.d, what=f"{case.name} tree {t} level {l}")
+
+
+@pytest.mark.parametrize("mode_i", [0, 1])
+def test_search_matches_oracle(case, mode_i):
+    w = case.w
+    if mode_i >= len(w.modes):
+        pytest.skip("workload has one mode")
+    mode, p, k = w.modes[mode_i]
+    Z = zha()
+    sel, cnt, st = case.tree.search(case.inp.Q, MODE[mode], p, k, with_stats=True)
+    case.tree.sync_status()
+    sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+    stats = Z.parse_stats(st)
+    ow = case.oracle_search(mode, p, k)
+    differ = compare_selection(sel, cnt, ow)
+    print(f"{case.name} {mode}: {len(differ)} of {len(ow)} walks part at oracle near-ties")
+    for wi, o in ow.items():
+        if wi in differ:
+            continue
+        s = stats[wi]
+        assert s["start_level"] == o.start_level
+        assert s["frontier"][: w.depth + 1][1:] == o.frontier[1:]
+        assert s["opened"][: w.depth + 1][1:] == o.opened[1:]
+        assert s["keys_read"] == o.keys_read and s["work"] == o.work
+
+
+def test_attend_on_oracle_selection(case):
+    w = case.w
+    mode, p, k = w.modes[0]
+    ow = case.oracle_search(mode, p, k)
+    n1 = case.otrees[(0, 0)].n_nodes[1]
+    W = w.walks
+    max_sel = max(1, max(len(o.sel) for o in ow.values()))
+    sel = np.zeros((W, max_sel), dtype=np.int32)
+    cnt = np.zeros(W, dtype=np.int32)
+    for wi, o in ow.items():
+        sel[wi, : len(o.sel)] = o.sel
+        cnt[wi] = len(o.sel)
+    sel_d, cnt_d = torch.from_numpy(sel).cuda(), torch.from_numpy(cnt).cuda()
+    out, lse = case.tree.attend(case.inp.Q, sel_d, cnt_d, out_dtype=torch.float32)
+    out_c, _ = case.tree.attend(case.inp.Q, sel_d, cnt_d)  # in the cache dtype
+    case.tree.sync_status()
+    out = host64(out).reshape(W, w.d)
+    out_c = host64(out_c).reshape(W, w.d)
+    lse = lse.cpu().numpy()
+    for wi, key, q in case.walks():
+        o_out, o_lse = O.attend(case.Kh[key], case.Vh[key], q, ow[wi].sel, w.chunk, n1, w.beta)
+        assert_attention_close(out[wi], lse[wi], o_out, o_lse, attn_tol(w), f"{case.name} walk {wi}")
+        if w.kv_dtype == "bf16":
+            assert_bf16_output_close(out_c[wi], o_out, f"{case.name} walk {wi}")
+
+
+def test_search_then_attend_end_to_end(case):
+    w = case.w
+    mode, p, k = w.modes[0]
+    sel, cnt, _ = case.tree.search(case.inp.Q, MODE[mode], p, k)
+    out, lse = case.tree.attend(case.inp.Q, sel, cnt, out_dtype=torch.float32)
+    case.tree.sync_status()
+    ow = case.oracle_search(mode, p, k)
+    differ = compare_selection(sel.cpu().numpy(), cnt.cpu().numpy(), ow)
+    out = host64(out).reshape(w.walks, w.d)
+    lse = lse.cpu().numpy()
+    n1 = case.otrees[(0, 0)].n_nodes[1]
+    for wi, key, q in case.walks():
+        if wi in differ:
+            continue
+        o_out, o_lse = O.attend(case.Kh[key], case.Vh[key], q, ow[wi].sel, w.chunk, n1, w.beta)
+        assert_attention_close(out[wi], lse[wi], o_out, o_lse, attn_tol(w), f"{case.name} walk {wi}")
+
+
+def test_p_one_is_dense_attention(case):
+    w = case.w
+    sel, cnt, _ = case.tree.search(case.inp.Q, O.TOP_P, 1.0, 0)
+    out, lse = case.tree.attend(case.inp.Q, sel, cnt, out_dtype=torch.float32)
+    case.tree.sync_status()
+    n1 = case.otrees[(0, 0)].n_nodes[1]
+    cnt = cnt.cpu().numpy()
+    assert (cnt == n1).all()
+    assert (sel.cpu().numpy()[:, :n1] == np.arange(n1)[None, :]).all()
+    out = host64(out).reshape(w.walks, w.d)
+    lse = lse.cpu().numpy()
+    for j, (wi, key, q) in enumerate(case.walks()):
+        if j % 7:
+            continue
+        Kd, Vd = case.Kh[key], case.Vh[key]
+        s = w.beta * Kd @ q
+        m = s.max()
+        e = np.exp(s - m)
+        ref = e @ Vd / e.sum()
+        assert_attention_close(out[wi], lse[wi], ref, m + np.log(e.sum()), attn_tol(w), f"{case.name} walk {wi}")
+
+
+# ---------------------------------------------------------------------------
+# edge cases, each against the oracle
+
+
+def _tiny(N, cap=None, C=8, depth=3, d=64, R=4, B=1, H=1, Hq=1, nq=4, dtype=torch.float32, seed=0):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    cap = cap or max(N, 1)
+    K = torch.randn(B, H, cap, d, generator=g, device="cuda").to(dtype)
+    V = torch.randn(B, H, cap, d, generator=g, device="cuda").to(dtype)
+    refs = torch.randn(H, R, d, generator=g, device="cuda")
+    Q = (2 * torch.randn(B, Hq, nq, d, generator=g, device="cuda")).to(dtype)
+    return K, V, refs, Q
+
+
+def _check_against_oracle(K, V, refs, Q, N, C, depth, beta, top_width=64, modes=((O.TOP_P, 0.9, 0),)):
+    Z = zha()
+    tree = Z.Tree(K, V, refs, N, C, depth, beta, top_width)
+    B, H, _, d = K.shape
+    Hq, nq = Q.shape[1], Q.shape[2]
+    group = Hq // H
+    R = refs.shape[1]
+    Qh = host64(Q)
+    for b in range(B):
+        for h in range(H):
+            ot = O.build_tree(host64(K[b, h, :N]), host64(refs[h]), C, depth, beta, store=O.STORE_F32)
+            for l in range(1, depth + 1):
+                g, n = gpu_level(tree, l, b * H + h)
+                assert n == ot.n_nodes[l]
+                if n:
+                    keys, bias = ot.level(l)
+                    assert_nodes_close(g, keys, bias, R, d)
+    for mode, p, k in modes:
+        sel, cnt, st = tree.search(Q, mode, p, k, max_sel=max(1, N // C), with_stats=True)
+        out, lse = tree.attend(Q, sel, cnt, out_dtype=torch.float32)
+        out_c, _ = tree.attend(Q, sel, cnt)
+        tree.sync_status()
+        sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+        stats = Z.parse_stats(st)
+        out = host64(out).reshape(-1, d)
+        out_c = host64(out_c).reshape(-1, d)
+        lse = lse.cpu().numpy()
+        for b in range(B):
+            for hq in range(Hq):
+                h = hq // group
+                ot = O.build_tree(host64(K[b, h, :N]), host64(refs[h]), C, depth, beta, store=O.STORE_F32)
+                Kd, Vd = host64(K[b, h, :N]), host64(V[b, h, :N])
+                for i in range(nq):
+                    wi = (b * Hq + hq) * nq + i
+                    ow = O.search(ot, Qh[b, hq, i], mode, p, k, top_width)
+                    compare_selection(sel, cnt, {wi: ow})
+                    if not np.array_equal(sel[wi, : cnt[wi]], ow.sel):
+                        continue
+                    assert stats[wi]["keys_read"] == ow.keys_read and stats[wi]["work"] == ow.work
+                    if N == 0:
+                        assert lse[wi] == -np.inf and not out[wi].any()
+                        continue
+                    o_out, o_lse = O.attend(Kd, Vd, Qh[b, hq, i], ow.sel, C, ot.n_nodes[1], beta)
+                    tol = 1e-5 if K.dtype == torch.float32 else 3e-3
+                    assert_attention_close(out[wi], lse[wi], o_out, o_lse, tol)
+                    if K.dtype == torch.bfloat16:
+                        assert_bf16_output_close(out_c[wi], o_out)
+    tree.close()
+
+
+ALL_MODES = ((O.TOP_P, 0.9, 0), (O.TOP_P, 1.0, 0), (O.TOP_P, 0.3, 0), (O.TOP_K, 0, 1), (O.TOP_K, 0, 3),
+             (O.TOP_K, 0, 1000))
+
+
+def test_tail_and_orphans():
+    # 1003 keys, C = 8: level sizes 125 / 15 / 1, five level-1 orphans, three tail keys
+    K, V, refs, Q = _tiny(1003, nq=6)
+    _check_against_oracle(K, V, refs, Q, 1003, 8, 3, 0.125, modes=ALL_MODES)
+
+
+def test_tree_smaller_than_a_chunk():
+    K, V, refs, Q = _tiny(5)
+    _check_against_oracle(K, V, refs, Q, 5, 8, 3, 0.125, modes=ALL_MODES)
+
+
+def test_empty_tree():
+    K, V, refs, Q = _tiny(0, cap=16)
+    _check_against_oracle(K, V, refs, Q, 0, 8, 2, 0.125)
+
+
+def test_walk_from_the_root():
+    K, V, refs, Q = _tiny(4096, C=4, depth=6, nq=8)
+    _check_against_oracle(K, V, refs, Q, 4096, 4, 6, 0.125, top_width=1, modes=ALL_MODES)
+
+
+def test_gqa_bf16_d128_and_d256():
+    for d in (128, 256):
+        K, V, refs, Q = _tiny(3000, C=16, depth=3, d=d, R=8, B=2, H=2, Hq=4, nq=3, dtype=torch.bfloat16, seed=d)
+        _check_against_oracle(K, V, refs, Q, 3000, 16, 3, 1 / np.sqrt(d), modes=ALL_MODES[:4])
+
+
+def test_odd_reference_count_and_chunk():
+    K, V, refs, Q = _tiny(2000, C=5, depth=4, d=64, R=3, nq=5)
+    _check_against_oracle(K, V, refs, Q, 2000, 5, 4, 0.2, modes=ALL_MODES)
+
+
+def test_max_sel_overflow_is_reported():
+    Z = zha()
+    K, V, refs, Q = _tiny(1024, C=8, depth=2)
+    tree = Z.Tree(K, V, refs, 1024, 8, 2, 0.125)
+    sel, cnt, _ = tree.search(Q, O.TOP_P, 1.0, 0, max_sel=3)
+    with pytest.raises(Z.ZhaError) as e:
+        tree.sync_status()
+    assert e.value.code == Z.ERR_CAPACITY
+    assert (cnt.cpu().numpy() == 3).all()
+    assert (sel.cpu().numpy() == np.arange(3)[None, :]).all()
+    tree.sync_status()  # cleared
+    tree.close()
+
+
+def test_append_equals_build():
+    Z = zha()
+    B, H, d, R, C, depth = 2, 2, 128, 8, 8, 4
+    N0, M = 1000, 1100
+    K, V, refs, Q = _tiny(N0 + M, C=C, depth=depth, d=d, R=R, B=B, H=H, Hq=4, nq=2, dtype=torch.bfloat16)
+    grown_K = K.clone()
+    grown_V = V.clone()
+    grown_K[:, :, N0:] = 0
+    grown_V[:, :, N0:] = 0
+    grown = Z.Tree(grown_K, grown_V, refs, N0, C, depth, 1 / np.sqrt(d))
+    for i in range(N0, N0 + M):
+        grown.append(K[:, :, i].contiguous(), V[:, :, i].contiguous())
+    assert grown.n_keys == N0 + M
+    assert torch.equal(grown_K, K) and torch.equal(grown_V, V)
+    direct = Z.Tree(K, V, refs, N0 + M, C, depth, 1 / np.sqrt(d))
+    assert grown.level_sizes() == direct.level_sizes() == [2100, 262, 32, 4, 0]
+    for l in range(1, depth + 1):
+        a, n = grown.level(l)
+        b, m = direct.level(l)
+        assert torch.equal(a[:, :n], b[:, :m])  # same kernel, same inputs: bit-identical
+    ot = O.build_tree(host64(K[1, 1, :N0]), host64(refs[1]), C, depth, 1 / np.sqrt(d), capacity=N0 + M)
+    O.append(ot, host64(K[1, 1]), M)
+    for l in range(1, depth + 1):
+        g, n = gpu_level(grown, l, 3)
+        if n:
+            assert_nodes_close(g, *ot.level(l), R, d)
+    grown.close()
+    direct.close()
+
+
+def test_append_past_capacity_is_refused():
+    Z = zha()
+    K, V, refs, Q = _tiny(64, C=8, depth=2)
+    tree = Z.Tree(K, V, refs, 64, 8, 2, 0.125)
+    with pytest.raises(Z.ZhaError) as e:
+        tree.append(K[:, :, 0].contiguous(), V[:, :, 0].contiguous())
+    assert e.value.code == Z.ERR_CAPACITY
+    tree.close()

@@ -1,0 +1,277 @@
+"""Python binding of libzha, the B200 (sm_100a) library for Zyphra Hierarchical
+Attention: a tree of compressed key summaries over a KV cache, walked top-down by
+each query, followed by attention over exactly the keys the walk chose.
+
+This module only marshals arguments (torch tensors -> device pointers, the current
+CUDA stream) into the C ABI declared in include/zha.h; every step runs in the
+library's CUDA kernels. There is no CPU fallback: without libzha.so or a CUDA
+device the calls raise.
+
+Names follow the C ABI: build / append / search / attend.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzha.so")
+MAX_DEPTH = 12
+
+OK, ERR_INVALID, ERR_CAPACITY, ERR_OOM, ERR_CUDA, ERR_INTERNAL, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5, -6
+F32, BF16 = 0, 1
+TOP_P, TOP_K = 0, 1
+
+# Every symbol include/zha.h declares.
+SYMBOLS = ("zha_build", "zha_append", "zha_search", "zha_attend", "zha_reserve", "zha_level",
+           "zha_num_keys", "zha_sync_status", "zha_destroy", "zha_last_error", "zha_version",
+           "zha_profile", "zha_profile_read", "zha_kernel_launches", "zha_last_search_info")
+KERNEL_KINDS = ("build", "append", "search_init", "score", "select", "attend_plan", "attend_partial",
+                "attend_combine")
+
+
+class ZhaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"zha error {code}: {msg}")
+        self.code = code
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("n_kv_heads", ctypes.c_int), ("d", ctypes.c_int),
+                ("R", ctypes.c_int), ("chunk", ctypes.c_int), ("depth", ctypes.c_int),
+                ("top_width", ctypes.c_int), ("capacity", ctypes.c_longlong),
+                ("sharpness", ctypes.c_float), ("kv_dtype", ctypes.c_int)]
+
+
+class Stats(ctypes.Structure):
+    _fields_ = [("start_level", ctypes.c_int), ("frontier", ctypes.c_int * (MAX_DEPTH + 1)),
+                ("opened", ctypes.c_int * (MAX_DEPTH + 1)), ("keys_read", ctypes.c_longlong),
+                ("work", ctypes.c_longlong)]
+
+
+STATS_BYTES = ctypes.sizeof(Stats)
+
+
+class KernelTime(ctypes.Structure):
+    _fields_ = [("launches", ctypes.c_longlong), ("ms", ctypes.c_double)]
+
+
+class SearchInfo(ctypes.Structure):
+    _fields_ = [("start_level", ctypes.c_int), ("union_nodes", ctypes.c_longlong * (MAX_DEPTH + 1)),
+                ("walk_nodes", ctypes.c_longlong * (MAX_DEPTH + 1))]
+
+_lib = None
+
+
+def lib():
+    """The loaded libzha.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run __graft_entry__.build() (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, ll, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
+        L.zha_build.argtypes = [ctypes.POINTER(Config), vp, vp, vp, ll, vp, ctypes.POINTER(vp)]
+        L.zha_append.argtypes = [vp, vp, vp, vp]
+        L.zha_search.argtypes = [vp, vp, i, i, i, i, f, i, vp, vp, i, vp, vp]
+        L.zha_attend.argtypes = [vp, vp, i, i, i, vp, vp, i, vp, i, vp, vp]
+        L.zha_reserve.argtypes = [vp, ll, i]
+        L.zha_level.argtypes = [vp, i, ctypes.POINTER(vp), ctypes.POINTER(ll), ctypes.POINTER(ll),
+                                ctypes.POINTER(i)]
+        L.zha_num_keys.argtypes = [vp]
+        L.zha_num_keys.restype = ll
+        L.zha_sync_status.argtypes = [vp, vp]
+        L.zha_destroy.argtypes = [vp]
+        L.zha_destroy.restype = None
+        L.zha_profile.argtypes = [vp, i]
+        L.zha_profile_read.argtypes = [vp, ctypes.POINTER(KernelTime), vp]
+        L.zha_kernel_launches.restype = ll
+        L.zha_kernel_launches.argtypes = []
+        L.zha_last_search_info.argtypes = [vp, ctypes.POINTER(SearchInfo), vp]
+        L.zha_last_error.restype = ctypes.c_char_p
+        L.zha_version.restype = ctypes.c_char_p
+        for name in SYMBOLS:
+            getattr(L, name)
+        _lib = L
+    return _lib
+
+
+def _check(rc: int):
+    if rc != OK:
+        raise ZhaError(rc, lib().zha_last_error().decode())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: use float32 or bfloat16")
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+class _DeviceArray:
+    """A non-owning __cuda_array_interface__ view of library-owned device memory."""
+
+    def __init__(self, ptr: int, shape, typestr: str, owner):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (ptr, False), "version": 3, "strides": None}
+        self._owner = owner
+
+
+class Tree:
+    """The summary trees of a KV cache [B][H_kv][capacity][d] (one per sequence and
+    KV head). K, V and refs stay referenced here: the library keeps their pointers."""
+
+    def __init__(self, K: torch.Tensor, V: torch.Tensor, refs: torch.Tensor, n_keys: int, chunk: int,
+                 depth: int, sharpness: float, top_width: int = 64, stream=None):
+        if K.dim() != 4 or V.shape != K.shape:
+            raise ValueError("K and V must both be [B][H_kv][capacity][d]")
+        if refs.dim() != 3 or refs.dtype != torch.float32 or refs.shape[0] != K.shape[1] or refs.shape[2] != K.shape[3]:
+            raise ValueError("refs must be fp32 [H_kv][R][d]")
+        if V.dtype != K.dtype:
+            raise ValueError("K and V must have the same dtype")
+        B, H, cap, d = K.shape
+        self.cfg = Config(batch=B, n_kv_heads=H, d=d, R=refs.shape[1], chunk=chunk, depth=depth,
+                          top_width=top_width, capacity=cap, sharpness=sharpness,
+                          kv_dtype=_dtype_code(K))
+        self.K, self.V, self.refs = K, V, refs
+        self._h = ctypes.c_void_p()
+        _check(lib().zha_build(ctypes.byref(self.cfg), _dev(K, "K"), _dev(V, "V"), _dev(refs, "refs"),
+                               int(n_keys), _stream(stream), ctypes.byref(self._h)))
+
+    # -- properties -------------------------------------------------------
+    @property
+    def handle(self) -> int:
+        return self._h.value
+
+    @property
+    def n_keys(self) -> int:
+        return int(lib().zha_num_keys(self._h))
+
+    def level_sizes(self) -> list:
+        out = [self.n_keys]
+        for l in range(1, self.cfg.depth + 1):
+            out.append(self.level(l)[1])
+        return out
+
+    def level(self, l: int):
+        """(nodes view [B*H_kv][level_capacity][node_floats] fp32, live node count)."""
+        ptr = ctypes.c_void_p()
+        n = ctypes.c_longlong()
+        cap = ctypes.c_longlong()
+        nf = ctypes.c_int()
+        _check(lib().zha_level(self._h, l, ctypes.byref(ptr), ctypes.byref(n), ctypes.byref(cap),
+                               ctypes.byref(nf)))
+        T = self.cfg.batch * self.cfg.n_kv_heads
+        if not ptr.value:
+            return torch.zeros(T, 0, nf.value, device=self.K.device), n.value
+        view = torch.as_tensor(_DeviceArray(ptr.value, (T, cap.value, nf.value), "<f4", self),
+                               device=self.K.device)
+        return view, n.value
+
+    # -- the hot path -----------------------------------------------------
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
+        B, H, _, d = self.K.shape
+        if k_new.shape != (B, H, d) or v_new.shape != (B, H, d) or k_new.dtype != self.K.dtype or v_new.dtype != self.K.dtype:
+            raise ValueError("k_new and v_new must be [B][H_kv][d] of the cache dtype")
+        _check(lib().zha_append(self._h, _dev(k_new, "k_new"), _dev(v_new, "v_new"), _stream(stream)))
+
+    def search(self, Q: torch.Tensor, mode: int = TOP_P, p: float = 0.9, k: int = 1, max_sel: int | None = None,
+               with_stats: bool = False, out=None, stream=None):
+        """Q: [B][H_q][n_q][d]. Returns (sel [walks][max_sel] int32, sel_count [walks] int32,
+        stats uint8 [walks][sizeof zha_stats] or None)."""
+        B, Hq, nq, d = Q.shape
+        W = B * Hq * nq
+        if max_sel is None:
+            max_sel = max(1, self.level(1)[1])
+        if out is None:
+            sel = torch.empty(W, max_sel, dtype=torch.int32, device=Q.device)
+            cnt = torch.empty(W, dtype=torch.int32, device=Q.device)
+            st = torch.empty(W, STATS_BYTES, dtype=torch.uint8, device=Q.device) if with_stats else None
+        else:
+            sel, cnt, st = out
+        _check(lib().zha_search(self._h, _dev(Q, "Q"), _dtype_code(Q), Hq, nq, mode, float(p), int(k),
+                                _dev(sel, "sel"), _dev(cnt, "sel_count"), max_sel,
+                                _dev(st, "stats") if st is not None else None, _stream(stream)))
+        return sel, cnt, st
+
+    def attend(self, Q: torch.Tensor, sel: torch.Tensor, sel_count: torch.Tensor, out=None, lse=None,
+               out_dtype=None, stream=None):
+        """Returns (out [B][H_q][n_q][d] of out_dtype (default: the cache dtype), lse [walks] fp32)."""
+        B, Hq, nq, d = Q.shape
+        W = B * Hq * nq
+        if out is None:
+            out = torch.empty(B, Hq, nq, d, dtype=out_dtype or self.K.dtype, device=Q.device)
+        if lse is None:
+            lse = torch.empty(W, dtype=torch.float32, device=Q.device)
+        _check(lib().zha_attend(self._h, _dev(Q, "Q"), _dtype_code(Q), Hq, nq, _dev(sel, "sel"),
+                                _dev(sel_count, "sel_count"), sel.shape[1], _dev(out, "out"), _dtype_code(out),
+                                _dev(lse, "lse"), _stream(stream)))
+        return out, lse
+
+    def reserve(self, max_walks: int, max_sel: int) -> None:
+        _check(lib().zha_reserve(self._h, int(max_walks), int(max_sel)))
+
+    # -- diagnostics --------------------------------------------------------
+    def profile(self, enable: bool) -> None:
+        _check(lib().zha_profile(self._h, 1 if enable else 0))
+
+    def profile_read(self, stream=None) -> dict:
+        arr = (KernelTime * len(KERNEL_KINDS))()
+        _check(lib().zha_profile_read(self._h, arr, _stream(stream)))
+        return {name: (arr[i].launches, arr[i].ms) for i, name in enumerate(KERNEL_KINDS)}
+
+    def last_search_info(self, stream=None) -> dict:
+        info = SearchInfo()
+        _check(lib().zha_last_search_info(self._h, ctypes.byref(info), _stream(stream)))
+        return {"start_level": info.start_level, "union_nodes": list(info.union_nodes),
+                "walk_nodes": list(info.walk_nodes)}
+
+    def sync_status(self, stream=None) -> None:
+        _check(lib().zha_sync_status(self._h, _stream(stream)))
+
+    def close(self) -> None:
+        if self._h and self._h.value:
+            lib().zha_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def parse_stats(st: torch.Tensor) -> list:
+    """Device stats bytes -> list of dicts (host)."""
+    raw = st.cpu().numpy().tobytes()
+    out = []
+    for w in range(st.shape[0]):
+        s = Stats.from_buffer_copy(raw[w * STATS_BYTES:(w + 1) * STATS_BYTES])
+        out.append({"start_level": s.start_level, "frontier": list(s.frontier), "opened": list(s.opened),
+                    "keys_read": s.keys_read, "work": s.work})
+    return out
+
+
+def kernel_launches() -> int:
+    """Kernels this library has launched in this process."""
+    return int(lib().zha_kernel_launches())
+
+
+def version() -> str:
+    return lib().zha_version().decode()

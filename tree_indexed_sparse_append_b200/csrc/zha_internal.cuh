@@ -1,0 +1,236 @@
+// Internal declarations shared by the CUDA translation units of libzha.
+// Nothing here is part of the public ABI (include/zha.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/zha.h"
+
+namespace zha {
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// Device-side error codes recorded in the tree's status word (first one wins).
+enum : int { DEV_OK = 0, DEV_CAPACITY = 1, DEV_BAD_INDEX = 2 };
+
+__device__ __forceinline__ void report(int *status, int code) {
+    if (status) atomicCAS(status, DEV_OK, code);
+}
+
+// ---------------------------------------------------------------------------
+// Loads. Node data is streamed once per launch: keep it out of L1.
+__device__ __forceinline__ float4 ld_stream4(const float *p) {
+    float4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p));
+    return v;
+}
+__device__ __forceinline__ float2 ld_stream2(const float *p) {
+    float2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint4 ld_stream_u4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// EPL consecutive floats owned by one lane.
+template <int EPL>
+__device__ __forceinline__ void load_f32(const float *p, float (&v)[EPL]) {
+    if constexpr (EPL == 2) {
+        float2 a = ld_stream2(p);
+        v[0] = a.x;
+        v[1] = a.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < EPL; i += 4) {
+            float4 a = ld_stream4(p + i);
+            v[i] = a.x;
+            v[i + 1] = a.y;
+            v[i + 2] = a.z;
+            v[i + 3] = a.w;
+        }
+    }
+}
+
+// EPL consecutive elements of T (float or bf16) as floats, through L1 (reused).
+template <int EPL>
+__device__ __forceinline__ void load_cached(const float *p, float (&v)[EPL]) {
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) v[i] = __ldg(p + i);
+}
+template <int EPL>
+__device__ __forceinline__ void load_cached(const __nv_bfloat16 *p, float (&v)[EPL]) {
+    // EPL bf16 = 2*EPL bytes, loaded as 32-bit words (2 elements each)
+    static_assert(EPL % 2 == 0, "bf16 lanes own an even number of columns");
+    const unsigned *w = reinterpret_cast<const unsigned *>(p);
+    unsigned u[EPL / 2];
+    if constexpr (EPL == 8) {
+        uint4 x = __ldg(reinterpret_cast<const uint4 *>(p));
+        u[0] = x.x; u[1] = x.y; u[2] = x.z; u[3] = x.w;
+    } else if constexpr (EPL == 4) {
+        uint2 x = __ldg(reinterpret_cast<const uint2 *>(p));
+        u[0] = x.x; u[1] = x.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < EPL / 2; ++i) u[i] = __ldg(w + i);
+    }
+#pragma unroll
+    for (int i = 0; i < EPL / 2; ++i) {
+        v[2 * i] = __uint_as_float(u[i] << 16);
+        v[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+    }
+}
+
+__device__ __forceinline__ float to_float(float x) { return x; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ void from_float(float x, float *p) { *p = x; }
+__device__ __forceinline__ void from_float(float x, __nv_bfloat16 *p) { *p = __float2bfloat16_rn(x); }
+
+// ---------------------------------------------------------------------------
+// Warp reductions.
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(FULL, x, o);
+    return x;
+}
+__device__ __forceinline__ double warp_sum(double x) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(FULL, x, o);
+    return x;
+}
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, o));
+    return x;
+}
+
+__host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+
+// Sums RP per-lane values across the warp so that afterwards every lane holds
+// one complete sum: that of row (lane >> (5 - log2 RP)). Each halving step
+// swaps half of the remaining values with the partner lane, so RP rows cost
+// RP - 1 + (5 - log2 RP) shuffles instead of 5 * RP.
+template <int RP>
+__device__ __forceinline__ float transpose_reduce(float (&v)[RP], int lane) {
+    constexpr int LG = ilog2(RP);
+#pragma unroll
+    for (int step = 0; step < LG; ++step) {
+        const int off = 16 >> step;
+        const int half = RP >> (step + 1);
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            float send = upper ? v[i] : v[i + half];
+            float keep = upper ? v[i + half] : v[i];
+            v[i] = keep + __shfl_xor_sync(FULL, send, off);
+        }
+    }
+    float x = v[0];
+#pragma unroll
+    for (int off = 16 >> LG; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
+    return x;
+}
+
+// ---------------------------------------------------------------------------
+// Monotone map of an fp32 score to an unsigned key (larger score, larger key).
+__device__ __forceinline__ uint32_t order_key(float s) {
+    uint32_t b = __float_as_uint(s);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+    uint32_t b = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+    return __uint_as_float(b);
+}
+
+// Frontier masses are summed as unsigned fixed point with 40 fractional bits:
+// the sums are exact and independent of the order of addition.
+constexpr double MASS_ONE = 1099511627776.0;  // 2^40
+__device__ __forceinline__ unsigned long long mass_fixed(float e) {
+    return (unsigned long long)__double2ull_rn((double)e * MASS_ONE);
+}
+
+}  // namespace zha
+
+// ---------------------------------------------------------------------------
+// Host side: the tree handle.
+struct zha_tree {
+    zha_config cfg;
+    int T;                                  // trees = batch * n_kv_heads
+    int NF;                                 // floats per node
+    int device;
+    long long n;                            // keys per tree
+    long long n_nodes[ZHA_MAX_DEPTH + 1];   // live nodes per tree, per level
+    long long cap_nodes[ZHA_MAX_DEPTH + 1]; // node capacity per tree, per level
+    float *nodes[ZHA_MAX_DEPTH + 1];        // [T][cap_nodes[l]][NF]
+    void *K;
+    void *V;
+    const float *refs;
+    int *d_status;
+
+    // scratch (grown on demand)
+    void *ws;
+    size_t ws_bytes;
+    long long ws_walks;
+    int ws_max_sel;
+
+    // diagnostics
+    struct zha_profiler *prof;  // NULL unless zha_profile(tree, 1)
+    long long last_W;
+    int last_G, last_start, last_max_sel;
+};
+
+namespace zha {
+
+// Scratch carved out of tree->ws for one search / attend of W walks.
+struct Scratch {
+    float *qf;                 // [W][D] queries as fp32
+    float *S;                  // [W][Sstride] node scores, indexed by node id
+    int *L[2];                 // [W][Lstride] frontier lists (ping-pong)
+    int *cnt[2];               // [W] frontier counts
+    unsigned *M[ZHA_MAX_DEPTH + 1];  // per level: [T][words_l][G] membership bits
+    unsigned *U[ZHA_MAX_DEPTH + 1];  // per level: [T][words_l] union bits
+    size_t M_bytes, U_bytes;
+    unsigned *M_base, *U_base;
+    int *item_off;             // [W + 1] attend items per walk (prefix)
+    float *partial;            // [max_items][D + 2]
+    long long Sstride, Lstride, max_items;
+};
+
+int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s);
+
+// kernel launchers (return cudaError_t of the launch)
+cudaError_t launch_build_level(const zha_tree *t, int level, long long j0, long long j1,
+                               cudaStream_t st);
+cudaError_t launch_append_kv(const zha_tree *t, const void *k_new, const void *v_new,
+                             cudaStream_t st);
+cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zha_dtype q_dtype,
+                          int G, long long W, int mode, float p, int k, int *sel, int *sel_count,
+                          int max_sel, zha_stats *stats, int start_level, cudaStream_t st);
+cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zha_dtype q_dtype,
+                          int G, long long W, const int *sel, const int *sel_count, int max_sel,
+                          void *out, zha_dtype out_dtype, float *lse, cudaStream_t st);
+
+int num_sms();
+
+// Every kernel launch is bracketed by probe_begin / probe_end: they count the
+// launch and, when the tree is being profiled, record a CUDA event pair.
+void probe_begin(const zha_tree *t, int kind, cudaStream_t st);
+void probe_end(const zha_tree *t, int kind, cudaStream_t st);
+
+struct Probe {
+    const zha_tree *t;
+    int kind;
+    cudaStream_t st;
+    Probe(const zha_tree *t_, int k, cudaStream_t s) : t(t_), kind(k), st(s) { probe_begin(t, kind, st); }
+    ~Probe() { probe_end(t, kind, st); }
+};
+
+}  // namespace zha

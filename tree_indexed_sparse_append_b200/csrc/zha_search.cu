@@ -1,0 +1,547 @@
+// Top-down walk of every query through its tree.
+//
+// Page "How does a tree of summaries search a context? How ZHA works":
+//   - section "What does a node summarize?": a node's score for a query q is
+//     max over references r of (beta * <key_r, q> + bias_r);
+//   - section "Run a small tree yourself" (route in tree.ts): the scores of the
+//     whole frontier of a walk go through one softmax; top-p opens the shortest
+//     prefix of the mass-ordered frontier holding at least p; the children of
+//     the opened nodes form the next frontier; opened level-1 nodes name the
+//     keys to read;
+//   - section "How does top-p differ from top-K?": top-K opens exactly K nodes.
+// Readings where the pages are silent: ties in mass go to the lower node id;
+// p >= 1 opens every node; nodes whose parent does not exist yet (orphans) join
+// their level's frontier; the walk starts at the lowest level with at most
+// top_width nodes.
+//
+// Design (one launch pair per level, no grid-wide synchronisation):
+//   score_level  Tree-major and load-balanced: a grid-stride loop over
+//                (tree, 4-node group) items of the union of the frontiers of the
+//                tree's walks (the GQA heads and queries that share the tree).
+//                Each node (R*d fp32 keys + R biases, 4 KB at R=8, d=128) is
+//                streamed from HBM once with 128-bit L1-bypassing loads and
+//                scored against every walk whose frontier holds it (a ballot over
+//                per-walk membership bits). Dot products reduce with a warp
+//                transpose-reduce (R rows in R-1+5-log2 R shuffles).
+//   select_level One CTA per walk. Exact selection without sorting: a 4-pass
+//                8-bit radix select over the fp32 score bits, where each bucket
+//                carries its count and its softmax mass in 40-bit fixed point
+//                (integer sums: exact and order-independent). Ties at the
+//                boundary score open in ascending node id. Opened nodes are
+//                compacted in id order by block scans; their children and the
+//                orphans of the level below form the next frontier (membership
+//                bits per walk and a per-tree union).
+#include <cmath>
+
+#include "zha_internal.cuh"
+
+namespace zha {
+namespace {
+
+constexpr int SEL_THREADS = 256;
+
+// ---------------------------------------------------------------------------
+// block-wide helpers for SEL_THREADS threads (8 warps)
+template <typename V>
+__device__ __forceinline__ V warp_incl_scan(V x, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        V y = __shfl_up_sync(FULL, x, o);
+        if (lane >= o) x += y;
+    }
+    return x;
+}
+
+// inclusive scan across the block; `sh` holds 8 + 1 values
+template <typename V>
+__device__ __forceinline__ V block_incl_scan(V x, V *sh, V *total) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    V inc = warp_incl_scan(x, lane);
+    if (lane == 31) sh[w] = inc;
+    __syncthreads();
+    if (w == 0) {
+        V s = lane < SEL_THREADS / 32 ? sh[lane] : V(0);
+        s = warp_incl_scan(s, lane);
+        if (lane < SEL_THREADS / 32) sh[lane] = s;
+    }
+    __syncthreads();
+    V base = w > 0 ? sh[w - 1] : V(0);
+    if (total) *total = sh[SEL_THREADS / 32 - 1];
+    __syncthreads();
+    return base + inc;
+}
+
+__device__ __forceinline__ float block_max(float x, float *sh) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    x = warp_max(x);
+    if (lane == 0) sh[w] = x;
+    __syncthreads();
+    float r = sh[0];
+#pragma unroll
+    for (int i = 1; i < SEL_THREADS / 32; ++i) r = fmaxf(r, sh[i]);
+    __syncthreads();
+    return r;
+}
+
+template <int EPL>
+__device__ __forceinline__ void load_q(const float *p, float (&v)[EPL]) {
+    if constexpr (EPL == 2) {
+        float2 a = __ldg(reinterpret_cast<const float2 *>(p));
+        v[0] = a.x;
+        v[1] = a.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < EPL; i += 4) {
+            float4 a = __ldg(reinterpret_cast<const float4 *>(p + i));
+            v[i] = a.x;
+            v[i + 1] = a.y;
+            v[i + 2] = a.z;
+            v[i + 3] = a.w;
+        }
+    }
+}
+
+// Sets bits [lo, hi) of one walk's membership row and of its tree's union.
+__device__ __forceinline__ void set_bits(unsigned *M_tree, unsigned *U_tree, int G, int g, long long lo,
+                                         long long hi) {
+    for (long long w = lo >> 5; w <= (hi - 1) >> 5; ++w) {
+        const long long b0 = lo > (w << 5) ? lo : (w << 5);
+        const long long b1 = hi < ((w + 1) << 5) ? hi : ((w + 1) << 5);
+        const int n = (int)(b1 - b0);
+        const unsigned mask = (n == 32 ? FULL : ((1u << n) - 1u)) << (int)(b0 - (w << 5));
+        atomicOr(&M_tree[w * G + g], mask);
+        atomicOr(&U_tree[w], mask);
+    }
+}
+
+// ---------------------------------------------------------------------------
+struct InitArgs {
+    const void *Q;
+    int q_bf16, D;
+    long long W;
+    float *qf;
+    int *n_par;           // frontier descriptor: parents opened (unused at the start level)
+    unsigned *M, *U;      // start level
+    long long words;
+    int G;
+    long long n_s;
+    zha_stats *stats;
+    int start_level;
+};
+
+__global__ void search_init_kernel(InitArgs a) {
+    const long long walk = blockIdx.x;
+    const int t = (int)(walk / a.G), g = (int)(walk % a.G);
+    for (int e = threadIdx.x; e < a.D; e += blockDim.x) {
+        const long long i = walk * a.D + e;
+        a.qf[i] = a.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16 *>(a.Q)[i])
+                           : static_cast<const float *>(a.Q)[i];
+    }
+    for (long long w = threadIdx.x; w < a.words; w += blockDim.x) {
+        const long long b0 = w << 5;
+        const long long n = a.n_s - b0;
+        const unsigned mask = n >= 32 ? FULL : (n <= 0 ? 0u : ((1u << n) - 1u));
+        a.M[((long long)t * a.words + w) * a.G + g] = mask;
+        if (g == 0) a.U[(long long)t * a.words + w] = mask;
+    }
+    if (threadIdx.x == 0) {
+        a.n_par[walk] = 0;
+        if (a.stats) {
+            zha_stats *s = a.stats + walk;
+            s->start_level = a.start_level;
+            for (int l = 0; l <= ZHA_MAX_DEPTH; ++l) s->frontier[l] = s->opened[l] = 0;
+            s->keys_read = 0;
+            s->work = 0;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+struct ScoreArgs {
+    const float *nodes;
+    long long node_tree;  // floats per tree in the level array
+    int NF, R, G, T;
+    float beta;
+    const unsigned *U, *M;
+    long long words, n_level;
+    const float *qf;
+    float *S;
+    long long Sstride;
+};
+
+template <int D, int RP>
+__global__ void __launch_bounds__(256) score_level_kernel(ScoreArgs a) {
+    constexpr int EPL = D / 32;
+    constexpr int LG = ilog2(RP);
+    const int lane = threadIdx.x & 31;
+    const int rr = lane >> (5 - LG);  // row whose full dot product this lane ends with
+    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+    const long long groups = (a.n_level + 3) >> 2;
+    const long long items = groups * a.T;
+
+    for (long long it = gw; it < items; it += nw) {
+        const int t = (int)(it / groups);
+        const long long j0 = (it - (long long)t * groups) << 2;
+        const unsigned word = a.U[(long long)t * a.words + (j0 >> 5)];
+        unsigned nib = (word >> (j0 & 31)) & 0xFu;
+        while (nib) {
+            const int b = __ffs(nib) - 1;
+            nib &= nib - 1;
+            const long long j = j0 + b;
+            const float *node = a.nodes + (long long)t * a.node_tree + j * a.NF;
+            float kr[RP][EPL];
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+                if (r < a.R) {
+                    load_f32<EPL>(node + r * D + lane * EPL, kr[r]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) kr[r][e] = 0.f;
+                }
+            }
+            const float bias = rr < a.R ? __ldg(node + a.R * D + rr) : 0.f;
+            const unsigned *Mrow = a.M + ((long long)t * a.words + (j >> 5)) * a.G;
+            const int bit = (int)(j & 31);
+            for (int g0 = 0; g0 < a.G; g0 += 32) {
+                const unsigned mw = (g0 + lane < a.G) ? __ldg(Mrow + g0 + lane) : 0u;
+                unsigned members = __ballot_sync(FULL, (mw >> bit) & 1u);
+                while (members) {
+                    const int gl = __ffs(members) - 1;
+                    members &= members - 1;
+                    const long long walk = (long long)t * a.G + g0 + gl;
+                    float q[EPL];
+                    load_q<EPL>(a.qf + walk * D + lane * EPL, q);
+                    float part[RP];
+#pragma unroll
+                    for (int r = 0; r < RP; ++r) {
+                        float s = 0.f;
+#pragma unroll
+                        for (int e = 0; e < EPL; ++e) s = fmaf(kr[r][e], q[e], s);
+                        part[r] = s;
+                    }
+                    const float dot = transpose_reduce<RP>(part, lane);
+                    float sc = rr < a.R ? fmaf(a.beta, dot, bias) : -INFINITY;
+#pragma unroll
+                    for (int off = 16; off >= (32 >> LG) && LG > 0; off >>= 1)
+                        sc = fmaxf(sc, __shfl_xor_sync(FULL, sc, off));
+                    if (lane == 0) a.S[walk * a.Sstride + j] = sc;
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+struct SelectArgs {
+    int level, C, R, G;
+    int start;               // 1 when this level is the start level (frontier = all nodes)
+    long long n_level;       // nodes at this level
+    long long n_orph;        // orphans at this level (nodes past C * n_{level+1}); 0 at start
+    long long n_orph_next;   // orphans at level - 1
+    long long n_level_next;  // nodes at level - 1 (for orphan ids)
+    const float *S;
+    long long Sstride;
+    const int *par_in;       // opened parents (level + 1), ascending
+    int *par_out;            // opened nodes of this level (when level > 1)
+    long long Lstride;
+    const int *n_par_in;
+    int *n_par_out;
+    unsigned *M_next, *U_next;
+    long long words_next;
+    int mode;
+    float p;
+    int k;
+    int *sel;
+    int max_sel;
+    int *sel_count;
+    zha_stats *stats;
+    long long tail;
+    int *status;
+};
+
+// frontier position -> node id
+__device__ __forceinline__ long long frontier_id(const SelectArgs &a, const int *par, long long npar,
+                                                 long long i) {
+    if (a.start) return i;
+    const long long kids = npar * a.C;
+    if (i < kids) return (long long)par[i / a.C] * a.C + i % a.C;
+    return (a.n_level - a.n_orph) + (i - kids);
+}
+
+__global__ void __launch_bounds__(SEL_THREADS) select_level_kernel(SelectArgs a) {
+    __shared__ unsigned long long h_mass[256];
+    __shared__ unsigned h_cnt[256];
+    __shared__ unsigned long long sh_u64[SEL_THREADS / 32];
+    __shared__ unsigned sh_u32[SEL_THREADS / 32];
+    __shared__ float sh_f[SEL_THREADS / 32];
+    __shared__ uint32_t s_prefix;
+    __shared__ unsigned long long s_trem;
+    __shared__ unsigned s_krem;
+
+    const long long walk = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int t = (int)(walk / a.G), g = (int)(walk % a.G);
+    const long long npar = a.start ? 0 : a.n_par_in[walk];
+    const int *par = a.par_in + walk * a.Lstride;
+    const long long F = a.start ? a.n_level : npar * a.C + a.n_orph;
+    const float *S = a.S + walk * a.Sstride;
+    const long long per = (F + SEL_THREADS - 1) / SEL_THREADS;
+    const long long beg = min(F, tid * per), end = min(F, beg + per);
+
+    const bool open_all = (a.mode == ZHA_TOP_P && a.p >= 1.f) || (a.mode == ZHA_TOP_K && (long long)a.k >= F);
+    uint32_t kstar = 0;
+    unsigned long long cstar = 0;
+    if (F > 0 && !open_all) {
+        float m = -INFINITY;
+        for (long long i = beg; i < end; ++i) m = fmaxf(m, S[frontier_id(a, par, npar, i)]);
+        m = block_max(m, sh_f);
+        unsigned long long trem = 0;
+        unsigned krem = (unsigned)a.k;
+        if (a.mode == ZHA_TOP_P) {
+            unsigned long long z = 0;
+            for (long long i = beg; i < end; ++i) z += mass_fixed(expf(S[frontier_id(a, par, npar, i)] - m));
+            unsigned long long Z;
+            block_incl_scan<unsigned long long>(z, sh_u64, &Z);
+            trem = (unsigned long long)ceil((double)a.p * (double)Z);
+            if (trem < 1) trem = 1;
+            if (trem > Z) trem = Z;
+        }
+        uint32_t prefix = 0, pmask = 0;
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            h_mass[tid] = 0;
+            h_cnt[tid] = 0;
+            __syncthreads();
+            for (long long i = beg; i < end; ++i) {
+                const float s = S[frontier_id(a, par, npar, i)];
+                const uint32_t key = order_key(s);
+                if ((key & pmask) == prefix) {
+                    const int b = (key >> shift) & 255;
+                    atomicAdd(&h_cnt[b], 1u);
+                    if (a.mode == ZHA_TOP_P) atomicAdd(&h_mass[b], mass_fixed(expf(s - m)));
+                }
+            }
+            __syncthreads();
+            const int b = 255 - tid;  // thread tid holds the tid-th bucket from the top
+            const unsigned long long vm = h_mass[b];
+            const unsigned vc = h_cnt[b];
+            const unsigned long long incl_m = block_incl_scan<unsigned long long>(vm, sh_u64, nullptr);
+            const unsigned incl_c = block_incl_scan<unsigned>(vc, sh_u32, nullptr);
+            const bool hit = a.mode == ZHA_TOP_P ? (incl_m - vm < trem && trem <= incl_m)
+                                                 : (incl_c - vc < krem && krem <= incl_c);
+            if (hit) {
+                s_prefix = prefix | ((uint32_t)b << shift);
+                s_trem = trem - (incl_m - vm);
+                s_krem = krem - (incl_c - vc);
+            }
+            __syncthreads();
+            prefix = s_prefix;
+            trem = s_trem;
+            krem = s_krem;
+            pmask |= 255u << shift;
+            __syncthreads();
+        }
+        kstar = prefix;
+        if (a.mode == ZHA_TOP_P) {
+            const unsigned long long u = mass_fixed(expf(key_to_float(kstar) - m));
+            cstar = u > 0 ? (trem + u - 1) / u : 1;
+        } else {
+            cstar = krem;
+        }
+    }
+
+    // opened = score key above kstar, or equal to it and among the first cstar (by id)
+    unsigned eq_local = 0;
+    if (!open_all)
+        for (long long i = beg; i < end; ++i)
+            eq_local += order_key(S[frontier_id(a, par, npar, i)]) == kstar;
+    unsigned eq_base = block_incl_scan<unsigned>(eq_local, sh_u32, nullptr) - eq_local;
+    unsigned open_local = 0;
+    {
+        unsigned eq = eq_base;
+        for (long long i = beg; i < end; ++i) {
+            bool o = open_all;
+            if (!open_all) {
+                const uint32_t key = order_key(S[frontier_id(a, par, npar, i)]);
+                o = key > kstar || (key == kstar && eq < cstar);
+                eq += key == kstar;
+            }
+            open_local += o;
+        }
+    }
+    unsigned n_open;
+    unsigned open_base = block_incl_scan<unsigned>(open_local, sh_u32, &n_open) - open_local;
+
+    // write the opened ids (ascending, since frontier positions ascend in id)
+    {
+        unsigned eq = eq_base, rank = open_base;
+        unsigned *M_tree = a.M_next ? a.M_next + (long long)t * a.words_next * a.G : nullptr;
+        unsigned *U_tree = a.U_next ? a.U_next + (long long)t * a.words_next : nullptr;
+        for (long long i = beg; i < end; ++i) {
+            const long long id = frontier_id(a, par, npar, i);
+            bool o = open_all;
+            if (!open_all) {
+                const uint32_t key = order_key(S[id]);
+                o = key > kstar || (key == kstar && eq < cstar);
+                eq += key == kstar;
+            }
+            if (!o) continue;
+            if (a.level == 1) {
+                if (rank < (unsigned)a.max_sel) a.sel[walk * a.max_sel + rank] = (int)id;
+            } else {
+                a.par_out[walk * a.Lstride + rank] = (int)id;
+                set_bits(M_tree, U_tree, a.G, g, id * a.C, id * a.C + a.C);
+            }
+            ++rank;
+        }
+        if (a.level > 1 && a.n_orph_next > 0) {
+            const long long lo = a.n_level_next - a.n_orph_next, hi = a.n_level_next;
+            for (long long w = (lo >> 5) + tid; w <= (hi - 1) >> 5; w += SEL_THREADS) {
+                const long long wlo = lo > (w << 5) ? lo : (w << 5);
+                const long long whi = hi < ((w + 1) << 5) ? hi : ((w + 1) << 5);
+                set_bits(M_tree, U_tree, a.G, g, wlo, whi);
+            }
+        }
+    }
+    if (tid == 0) {
+        if (a.level > 1) {
+            a.n_par_out[walk] = (int)n_open;
+        } else {
+            a.sel_count[walk] = (int)min(n_open, (unsigned)a.max_sel);
+            if (n_open > (unsigned)a.max_sel) report(a.status, DEV_CAPACITY);
+        }
+        if (a.stats) {
+            zha_stats *s = a.stats + walk;
+            s->frontier[a.level] = (int)F;
+            s->opened[a.level] = (int)n_open;
+            if (a.level == 1) {
+                long long sum = 0;
+                for (int l = 1; l <= ZHA_MAX_DEPTH; ++l) sum += s->frontier[l];
+                s->keys_read = (long long)a.C * n_open + a.tail;
+                s->work = (long long)a.R * sum + s->keys_read;
+            }
+        }
+    }
+}
+
+template <int D, int RP>
+cudaError_t launch_score(const zha_tree *t, const ScoreArgs &a, cudaStream_t st) {
+    const long long items = ((a.n_level + 3) >> 2) * a.T;
+    long long blocks = (items + 7) / 8;
+    const long long cap = (long long)num_sms() * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) return cudaSuccess;
+    Probe pr(t, ZHA_K_SCORE, st);
+    score_level_kernel<D, RP><<<(unsigned)blocks, 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_score_d(const zha_tree *t, const ScoreArgs &a, cudaStream_t st) {
+    if (a.R <= 1) return launch_score<D, 1>(t, a, st);
+    if (a.R <= 2) return launch_score<D, 2>(t, a, st);
+    if (a.R <= 4) return launch_score<D, 4>(t, a, st);
+    if (a.R <= 8) return launch_score<D, 8>(t, a, st);
+    return launch_score<D, 16>(t, a, st);
+}
+
+}  // namespace
+
+cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zha_dtype q_dtype, int G,
+                          long long W, int mode, float p, int k, int *sel, int *sel_count, int max_sel,
+                          zha_stats *stats, int start_level, cudaStream_t st) {
+    const zha_config &c = t->cfg;
+    const int D = c.d, C = c.chunk;
+    cudaError_t e;
+    if (s.M_bytes) {
+        e = cudaMemsetAsync(s.M_base, 0, s.M_bytes, st);
+        if (e != cudaSuccess) return e;
+        e = cudaMemsetAsync(s.U_base, 0, s.U_bytes, st);
+        if (e != cudaSuccess) return e;
+    }
+    auto words = [&](int l) { return (t->cap_nodes[l] + 31) / 32; };
+
+    InitArgs ia;
+    ia.Q = Q;
+    ia.q_bf16 = q_dtype == ZHA_BF16;
+    ia.D = D;
+    ia.W = W;
+    ia.qf = s.qf;
+    ia.n_par = s.cnt[0];
+    ia.M = s.M[start_level];
+    ia.U = s.U[start_level];
+    ia.words = words(start_level);
+    ia.G = G;
+    ia.n_s = t->n_nodes[start_level];
+    ia.stats = stats;
+    ia.start_level = start_level;
+    {
+        Probe pr(t, ZHA_K_SEARCH_INIT, st);
+        search_init_kernel<<<(unsigned)W, 128, 0, st>>>(ia);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+
+    int cur = 0;
+    for (int l = start_level; l >= 1; --l) {
+        ScoreArgs sa;
+        sa.nodes = t->nodes[l];
+        sa.node_tree = t->cap_nodes[l] * t->NF;
+        sa.NF = t->NF;
+        sa.R = c.R;
+        sa.G = G;
+        sa.T = t->T;
+        sa.beta = c.sharpness;
+        sa.U = s.U[l];
+        sa.M = s.M[l];
+        sa.words = words(l);
+        sa.n_level = t->n_nodes[l];
+        sa.qf = s.qf;
+        sa.S = s.S;
+        sa.Sstride = s.Sstride;
+        switch (D) {
+            case 64: e = launch_score_d<64>(t, sa, st); break;
+            case 128: e = launch_score_d<128>(t, sa, st); break;
+            default: e = launch_score_d<256>(t, sa, st); break;
+        }
+        if (e != cudaSuccess) return e;
+
+        SelectArgs se;
+        se.level = l;
+        se.C = C;
+        se.R = c.R;
+        se.G = G;
+        se.start = l == start_level;
+        se.n_level = t->n_nodes[l];
+        se.n_orph = l == start_level ? 0 : t->n_nodes[l] - (long long)C * t->n_nodes[l + 1];
+        se.n_level_next = l > 1 ? t->n_nodes[l - 1] : 0;
+        se.n_orph_next = l > 1 ? t->n_nodes[l - 1] - (long long)C * t->n_nodes[l] : 0;
+        se.S = s.S;
+        se.Sstride = s.Sstride;
+        se.par_in = s.L[cur];
+        se.par_out = s.L[cur ^ 1];
+        se.Lstride = s.Lstride;
+        se.n_par_in = s.cnt[cur];
+        se.n_par_out = s.cnt[cur ^ 1];
+        se.M_next = l > 1 ? s.M[l - 1] : nullptr;
+        se.U_next = l > 1 ? s.U[l - 1] : nullptr;
+        se.words_next = l > 1 ? words(l - 1) : 0;
+        se.mode = mode;
+        se.p = p;
+        se.k = k;
+        se.sel = sel;
+        se.max_sel = max_sel;
+        se.sel_count = sel_count;
+        se.stats = stats;
+        se.tail = t->n - (long long)C * t->n_nodes[1];
+        se.status = t->d_status;
+        {
+            Probe pr(t, ZHA_K_SELECT, st);
+            select_level_kernel<<<(unsigned)W, SEL_THREADS, 0, st>>>(se);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        cur ^= 1;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace zha
