@@ -131,6 +131,23 @@ class Clocks:
 
 
 # ---------------------------------------------------------------------------
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Largest value over the ranks (the slowest rank's time); no-op at world 1."""
+    if world <= 1:
+        return float(value)
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(walks_per_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job queries/s: every rank ran `steps` steps of `walks_per_step` walks;
+    the job took as long as its slowest rank."""
+    return walks_per_step * steps * world / (max_ms / 1e3)
+
+
 def oracle_walks_per_second(w, trees, seconds: float, cores: int):
     """Oracle (CPU) append + search + attend over the sampled trees' walks,
     repeated for about `seconds`; returns (queries/s, walks timed)."""
@@ -188,7 +205,7 @@ def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes
     import tree_indexed_sparse_append_b200 as Z
 
     steps, warmup = args.steps, args.warmup
-    need = warmup + steps + args.profile_steps + args.e2e_steps + 8
+    need = len(modes) * (warmup + steps + args.profile_steps) + args.e2e_steps + 8
     w = S.scaled(w, seed=w.seed + 7919 * rank, appends=max(w.appends, need))
     inp = S.draw(w, device="cuda")
     st = torch.cuda.current_stream()
@@ -240,13 +257,10 @@ def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes
             torch.cuda.synchronize()
         launches = Z.kernel_launches() - launches0
         tree.sync_status()
-        total_ms = sum(a.elapsed_time(b) for a, b in evs)
+        total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world, dev)
         if world > 1:
-            t = torch.tensor([total_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            total_ms = float(t.item())
             torch.distributed.barrier()
-        qps = Wk * steps * world / (total_ms / 1e3)
+        qps = job_throughput(Wk, steps, world, total_ms)
 
         # profiled pass: per-kernel device time and the frontier sizes behind it
         tree.profile(True)
@@ -323,13 +337,9 @@ def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes
         lse_h.copy_(lse, non_blocking=True)
     eb.record(st)
     torch.cuda.synchronize()
-    e2e_ms = ea.elapsed_time(eb)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(ea.elapsed_time(eb), world, dev)
     elt = inp.K.element_size()
-    e2e = {"value": Wk * args.e2e_steps * world / (e2e_ms / 1e3), "unit": UNIT,
+    e2e = {"value": job_throughput(Wk, args.e2e_steps, world, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": Qd.numel() * Qd.element_size() + 2 * kd.numel() * elt,
            "d2h_bytes_per_step": out.numel() * out.element_size() + lse.numel() * 4}
 

@@ -9,9 +9,10 @@ Tolerances (per element g = GPU, o = oracle):
       absolute error of a few ulps of the row, not of itself;
   attention outputs (fp32) and lse: |g - o| <= atol * max(1, |o|), atol = 1e-5
       for an fp32 cache and 3e-3 for a bf16 cache;
-  attention outputs stored as bf16: within one bf16 ulp of the oracle's output
-      rounded to bf16 (rounding alone moves a value by up to 2^-8 relative, more
-      than 3e-3, and values near a rounding boundary may round either way);
+  attention outputs stored as bf16: |g - o| <= half a bf16 ulp (the rounding of
+      the stored value) + 1e-5 * max(1, max|o| over the output row) (the fp32
+      arithmetic before rounding); rounding alone moves a value by up to 2^-9
+      relative, so the 3e-3 target is checked on the fp32 output;
   selected chunk sets: identical, unless the oracle's walk met a near-tie: a
       relative gap below 1e-5 between the last opened and the first unopened
       mass, or a running top-p sum within 1e-5 * p of p.
@@ -82,21 +83,15 @@ def compare_selection(sel: np.ndarray, cnt: np.ndarray, walks: dict):
     return differ
 
 
-def bf16_round(x: np.ndarray) -> np.ndarray:
-    import torch as _t
-
-    return _t.from_numpy(np.asarray(x, dtype=np.float32)).to(_t.bfloat16).to(_t.float64).numpy()
-
-
 def bf16_ulp(x: np.ndarray) -> np.ndarray:
     e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -126)))
     return 2.0 ** (e - 7)
 
 
 def assert_bf16_output_close(out_g: np.ndarray, out_o: np.ndarray, what: str = ""):
-    r = bf16_round(out_o)
-    bad = np.abs(out_g - r) > bf16_ulp(r) * 1.0001
-    assert not bad.any(), f"{what}: {bad.sum()} bf16 outputs more than one ulp from the rounded oracle"
+    allow = 0.5 * bf16_ulp(np.maximum(np.abs(out_g), np.abs(out_o))) + 1e-5 * max(1.0, np.abs(out_o).max())
+    bad = np.abs(out_g - out_o) > allow
+    assert not bad.any(), f"{what}: {bad.sum()} bf16 outputs off by more than half an ulp"
 
 
 def assert_attention_close(out_g: np.ndarray, lse_g: float, out_o: np.ndarray, lse_o: float, atol: float,

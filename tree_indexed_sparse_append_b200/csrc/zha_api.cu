@@ -142,9 +142,11 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     (void)G;
     const long long cap1 = t->cap_nodes[1] > 0 ? t->cap_nodes[1] : 1;
     const long long cap2 = c.depth >= 2 && t->cap_nodes[2] > 0 ? t->cap_nodes[2] : 1;
+    // attend items: a walk's keys (at most C * (max_sel + 1)) in items of >= 64 keys,
+    // at most 128 items per walk (constants of zha_attend.cu)
     const long long keys_max = (long long)c.chunk * ((long long)max_sel + 1);
-    long long per_walk_items = (keys_max + 127) / 128;
-    if (per_walk_items > 64) per_walk_items = 64;
+    long long per_walk_items = (keys_max + 63) / 64;
+    if (per_walk_items > 128) per_walk_items = 128;
     if (per_walk_items < 1) per_walk_items = 1;
     const long long max_items = W * per_walk_items;
 
@@ -169,6 +171,7 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     for (int l = 1; l <= c.depth; ++l) o_U[l] = take(sizeof(unsigned) * t->T * ((t->cap_nodes[l] + 31) / 32));
     const size_t U_bytes = off - U_start;
     const size_t o_io = take(sizeof(int) * (W + 1));
+    const size_t o_iw = take(sizeof(int) * max_items);
     const size_t o_pa = take(sizeof(float) * max_items * (c.d + 2));
     const size_t need = off;
 
@@ -199,6 +202,7 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     s->M_bytes = M_bytes;
     s->U_bytes = U_bytes;
     s->item_off = reinterpret_cast<int *>(b + o_io);
+    s->item_walk = reinterpret_cast<int *>(b + o_iw);
     s->partial = reinterpret_cast<float *>(b + o_pa);
     s->Sstride = cap1;
     s->Lstride = cap2;

@@ -8,14 +8,16 @@
 // with the same scale beta as the summaries.
 //
 // Design (split-K decode attention, fp32 accumulation):
-//   attend_plan     one CTA scans the walks' key counts into item offsets; a
-//                   walk's key list is cut into at most MAX_SPLIT items of at
-//                   least SEG keys.
-//   attend_partial  grid-stride over items, one warp per item. A row of K or V
-//                   is read with 16-byte loads by LPR lanes (16 for d = 128
-//                   bf16), so a warp handles 32/LPR keys per step; keys of one
-//                   selected chunk are contiguous in the cache. Online softmax
-//                   per lane group, merged across groups at the end; fp32 caches
+//   attend_plan     one CTA scans the walks' key counts into item offsets and an
+//                   item -> walk map; a walk's key list is cut into at most
+//                   MAX_SPLIT items of at least SEG keys.
+//   attend_partial  grid-stride over items, one warp per item. The item's chunk
+//                   ids are loaded once (one per lane) and broadcast by shuffle.
+//                   A row of K or V is read with 16-byte loads by LPR lanes (16
+//                   for d = 128 bf16), so a warp step covers 32/LPR keys, and
+//                   UNROLL steps of rows are in flight before any is used; keys
+//                   of one chunk are contiguous in the cache. Online softmax per
+//                   lane group, merged across groups at the end; fp32 caches
 //                   take their dot products in fp64.
 //   attend_combine  one warp per walk merges its items by log-sum-exp.
 #include <cmath>
@@ -26,8 +28,9 @@
 namespace zha {
 namespace {
 
-constexpr int SEG = 128;
-constexpr int MAX_SPLIT = 64;
+constexpr int SEG = 64;         // keys per work item, at least
+constexpr int MAX_SPLIT = 128;  // work items per walk, at most
+constexpr int UNROLL = 4;       // key groups whose rows are in flight together
 
 __device__ __forceinline__ long long walk_keys(const int *sel_count, long long w, int max_sel, int C,
                                                long long tail) {
@@ -46,6 +49,7 @@ struct PlanArgs {
     int max_sel, C;
     long long tail, W;
     int *item_off;
+    int *item_walk;
 };
 
 __global__ void __launch_bounds__(1024) attend_plan_kernel(PlanArgs a) {
@@ -78,7 +82,10 @@ __global__ void __launch_bounds__(1024) attend_plan_kernel(PlanArgs a) {
         }
         __syncthreads();
         const long long excl = carry + (wid > 0 ? sh[wid - 1] : 0) + inc - items;
-        if (w < a.W) a.item_off[w] = (int)excl;
+        if (w < a.W) {
+            a.item_off[w] = (int)excl;
+            for (long long i = 0; i < items; ++i) a.item_walk[excl + i] = (int)w;
+        }
         carry += sh[(blockDim.x >> 5) - 1];
         __syncthreads();
     }
@@ -88,7 +95,7 @@ __global__ void __launch_bounds__(1024) attend_plan_kernel(PlanArgs a) {
 struct PartialArgs {
     const void *K, *V, *Q;
     int q_bf16;
-    const int *sel, *sel_count, *item_off;
+    const int *sel, *sel_count, *item_off, *item_walk;
     int max_sel, C, G;
     long long W, cap, n1, tail;
     float beta;
@@ -142,20 +149,21 @@ __global__ void __launch_bounds__(256) attend_partial_kernel(PartialArgs a) {
     const T *Vb = static_cast<const T *>(a.V);
 
     for (long long item = gw; item < total; item += nw) {
-        // walk of this item: last w with item_off[w] <= item
-        long long lo = 0, hi = a.W;  // item_off[lo] <= item < item_off[hi]
-        while (hi - lo > 1) {
-            const long long mid = (lo + hi) >> 1;
-            if (a.item_off[mid] <= item) lo = mid;
-            else hi = mid;
-        }
-        const long long walk = lo;
+        const long long walk = a.item_walk[item];
         const long long tree = walk / a.G;
         const long long L = walk_keys(a.sel_count, walk, a.max_sel, a.C, a.tail);
         const long long seg = seg_len(L);
         const long long k0 = (item - a.item_off[walk]) * seg;
         const long long k1 = k0 + seg < L ? k0 + seg : L;
         const long long nsel = L - a.tail;  // keys coming from selected chunks
+        const int *wsel = a.sel + walk * a.max_sel;
+
+        // the segment's chunk ids, one per lane, when they fit in a warp
+        const long long c0 = k0 / a.C;
+        const long long c1 = (k1 < nsel ? k1 : nsel) > k0 ? ((k1 < nsel ? k1 : nsel) - 1) / a.C + 1 : c0;
+        const bool pre = c1 - c0 <= 32;
+        int my_chunk = 0;
+        if (pre && c0 + lane < c1) my_chunk = __ldg(wsel + c0 + lane);
 
         float q[COLS];
 #pragma unroll
@@ -171,44 +179,61 @@ __global__ void __launch_bounds__(256) attend_partial_kernel(PartialArgs a) {
 #pragma unroll
         for (int c = 0; c < COLS; ++c) acc[c] = 0.f;
 
-        for (long long kb = k0; kb < k1; kb += KPW) {
-            const long long kk = kb + grp;
-            bool valid = kk < k1;
-            long long kid = 0;
-            if (valid) {
-                if (kk < nsel) {
-                    const int c = __ldg(a.sel + walk * a.max_sel + kk / a.C);
-                    if (c < 0 || c >= a.n1) {
-                        valid = false;
-                        if (gl == 0) report(a.status, DEV_BAD_INDEX);
+        for (long long kb = k0; kb < k1; kb += KPW * UNROLL) {
+            bool valid[UNROLL];
+            long long kid[UNROLL];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const long long kk = kb + u * KPW + grp;
+                valid[u] = kk < k1;
+                kid[u] = 0;
+                int c = 0;
+                if (pre) {
+                    const long long src = kk < nsel ? kk / a.C - c0 : 0;
+                    c = __shfl_sync(FULL, my_chunk, (int)(src & 31));
+                } else if (valid[u] && kk < nsel) {
+                    c = __ldg(wsel + kk / a.C);
+                }
+                if (valid[u]) {
+                    if (kk < nsel) {
+                        if (c < 0 || c >= a.n1) {
+                            valid[u] = false;
+                            if (gl == 0) report(a.status, DEV_BAD_INDEX);
+                        } else {
+                            kid[u] = (long long)c * a.C + kk % a.C;
+                        }
                     } else {
-                        kid = (long long)c * a.C + kk % a.C;
+                        kid[u] = a.n1 * a.C + (kk - nsel);
                     }
-                } else {
-                    kid = a.n1 * a.C + (kk - nsel);
                 }
             }
-            const long long row = (tree * a.cap + kid) * D;
-            float kf[COLS], vf[COLS];
+            float kf[UNROLL][COLS], vf[UNROLL][COLS];
 #pragma unroll
-            for (int v = 0; v < VPL; ++v) {
-                Row<T>::load(Kb + row + (v * LPR + gl) * EPL, kf + v * EPL);
-                Row<T>::load(Vb + row + (v * LPR + gl) * EPL, vf + v * EPL);
+            for (int u = 0; u < UNROLL; ++u) {
+                const long long row = (tree * a.cap + kid[u]) * D;
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) {
+                    Row<T>::load(Kb + row + (v * LPR + gl) * EPL, kf[u] + v * EPL);
+                    Row<T>::load(Vb + row + (v * LPR + gl) * EPL, vf[u] + v * EPL);
+                }
             }
-            Dot d = 0;
 #pragma unroll
-            for (int c = 0; c < COLS; ++c) d += (Dot)kf[c] * (Dot)q[c];
+            for (int u = 0; u < UNROLL; ++u) {
+                Dot d = 0;
 #pragma unroll
-            for (int o = LPR / 2; o >= 1; o >>= 1) d += __shfl_xor_sync(FULL, d, o);
-            const float s = (float)((Dot)a.beta * d);
-            if (valid) {
-                const float mn = fmaxf(m, s);
-                const float scale = expf(m - mn);
-                const float pw = expf(s - mn);
-                l = l * scale + pw;
+                for (int c = 0; c < COLS; ++c) d += (Dot)kf[u][c] * (Dot)q[c];
 #pragma unroll
-                for (int c = 0; c < COLS; ++c) acc[c] = fmaf(pw, vf[c], acc[c] * scale);
-                m = mn;
+                for (int o = LPR / 2; o >= 1; o >>= 1) d += __shfl_xor_sync(FULL, d, o);
+                const float s = (float)((Dot)a.beta * d);
+                if (valid[u]) {
+                    const float mn = fmaxf(m, s);
+                    const float scale = expf(m - mn);
+                    const float pw = expf(s - mn);
+                    l = l * scale + pw;
+#pragma unroll
+                    for (int c = 0; c < COLS; ++c) acc[c] = fmaf(pw, vf[u][c], acc[c] * scale);
+                    m = mn;
+                }
             }
         }
         // merge the KPW lane groups
@@ -309,13 +334,14 @@ cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zh
                           long long W, const int *sel, const int *sel_count, int max_sel, void *out,
                           zha_dtype out_dtype, float *lse, cudaStream_t st) {
     const zha_config &c = t->cfg;
-    PlanArgs pl;
+    PlanArgs pl{};
     pl.sel_count = sel_count;
     pl.max_sel = max_sel;
     pl.C = c.chunk;
     pl.tail = t->n - (long long)c.chunk * t->n_nodes[1];
     pl.W = W;
     pl.item_off = s.item_off;
+    pl.item_walk = s.item_walk;
     {
         Probe pr(t, ZHA_K_ATTEND_PLAN, st);
         attend_plan_kernel<<<1, 1024, 0, st>>>(pl);
@@ -323,7 +349,7 @@ cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zh
         if (e != cudaSuccess) return e;
     }
 
-    PartialArgs pa;
+    PartialArgs pa{};
     pa.K = t->K;
     pa.V = t->V;
     pa.Q = Q;
@@ -331,6 +357,7 @@ cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zh
     pa.sel = sel;
     pa.sel_count = sel_count;
     pa.item_off = s.item_off;
+    pa.item_walk = s.item_walk;
     pa.max_sel = max_sel;
     pa.C = c.chunk;
     pa.G = G;
@@ -341,7 +368,7 @@ cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zh
     pa.beta = c.sharpness;
     pa.partial = s.partial;
     pa.status = t->d_status;
-    CombineArgs ca;
+    CombineArgs ca{};
     ca.item_off = s.item_off;
     ca.partial = s.partial;
     ca.W = W;

@@ -149,7 +149,7 @@ cudaError_t launch_build_level(const zha_tree *t, int level, long long j0, long 
                                cudaStream_t st) {
     if (j1 <= j0) return cudaSuccess;
     const zha_config &c = t->cfg;
-    BuildArgs a;
+    BuildArgs a{};
     a.refs = t->refs;
     a.out = t->nodes[level];
     a.out_tree = t->cap_nodes[level] * t->NF;

@@ -200,6 +200,7 @@ struct Scratch {
     size_t M_bytes, U_bytes;
     unsigned *M_base, *U_base;
     int *item_off;             // [W + 1] attend items per walk (prefix)
+    int *item_walk;            // [max_items] walk of each attend item
     float *partial;            // [max_items][D + 2]
     long long Sstride, Lstride, max_items;
 };

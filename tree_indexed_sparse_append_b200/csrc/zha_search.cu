@@ -31,6 +31,7 @@
 //                compacted in id order by block scans; their children and the
 //                orphans of the level below form the next frontier (membership
 //                bits per walk and a per-tree union).
+#include <algorithm>
 #include <cmath>
 
 #include "zha_internal.cuh"
@@ -69,18 +70,6 @@ __device__ __forceinline__ V block_incl_scan(V x, V *sh, V *total) {
     if (total) *total = sh[SEL_THREADS / 32 - 1];
     __syncthreads();
     return base + inc;
-}
-
-__device__ __forceinline__ float block_max(float x, float *sh) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    x = warp_max(x);
-    if (lane == 0) sh[w] = x;
-    __syncthreads();
-    float r = sh[0];
-#pragma unroll
-    for (int i = 1; i < SEL_THREADS / 32; ++i) r = fmaxf(r, sh[i]);
-    __syncthreads();
-    return r;
 }
 
 template <int EPL>
@@ -258,6 +247,7 @@ struct SelectArgs {
     zha_stats *stats;
     long long tail;
     int *status;
+    long long smem_keys;     // frontiers up to this size are staged in shared memory
 };
 
 // frontier position -> node id
@@ -269,15 +259,37 @@ __device__ __forceinline__ long long frontier_id(const SelectArgs &a, const int 
     return (a.n_level - a.n_orph) + (i - kids);
 }
 
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t x, unsigned *sh) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x = max(x, __shfl_xor_sync(FULL, x, o));
+    if (lane == 0) sh[w] = x;
+    __syncthreads();
+    uint32_t r = sh[0];
+#pragma unroll
+    for (int i = 1; i < SEL_THREADS / 32; ++i) r = max(r, sh[i]);
+    __syncthreads();
+    return r;
+}
+
+// Each walk's frontier keys are staged once in shared memory (up to
+// SEL_SMEM_KEYS of them; larger frontiers are re-read from the score array).
+// Histograms are kept in HCOPIES copies (warp w uses copy w % HCOPIES) so that
+// lanes with equal top bits contend less.
+constexpr int SEL_SMEM_KEYS = 8192;
+constexpr int HCOPIES = 4;
+
 __global__ void __launch_bounds__(SEL_THREADS) select_level_kernel(SelectArgs a) {
-    __shared__ unsigned long long h_mass[256];
-    __shared__ unsigned h_cnt[256];
+    extern __shared__ uint32_t skey[];
+    __shared__ unsigned long long h_mass[HCOPIES][256];
+    __shared__ unsigned h_cnt[HCOPIES][256];
+    __shared__ unsigned h_max[HCOPIES][256];
     __shared__ unsigned long long sh_u64[SEL_THREADS / 32];
     __shared__ unsigned sh_u32[SEL_THREADS / 32];
-    __shared__ float sh_f[SEL_THREADS / 32];
     __shared__ uint32_t s_prefix;
     __shared__ unsigned long long s_trem;
     __shared__ unsigned s_krem;
+    __shared__ int s_done;
 
     const long long walk = blockIdx.x;
     const int tid = threadIdx.x;
@@ -286,75 +298,104 @@ __global__ void __launch_bounds__(SEL_THREADS) select_level_kernel(SelectArgs a)
     const int *par = a.par_in + walk * a.Lstride;
     const long long F = a.start ? a.n_level : npar * a.C + a.n_orph;
     const float *S = a.S + walk * a.Sstride;
-    const long long per = (F + SEL_THREADS - 1) / SEL_THREADS;
-    const long long beg = min(F, tid * per), end = min(F, beg + per);
+    const bool staged = F <= a.smem_keys;
+    auto key_at = [&](long long i) -> uint32_t {
+        return staged ? skey[i] : order_key(S[frontier_id(a, par, npar, i)]);
+    };
+
+    // stage the frontier's keys (coalesced, strided) and find the largest
+    uint32_t kmax = 0;
+    for (long long i = tid; i < F; i += SEL_THREADS) {
+        const uint32_t k = order_key(S[frontier_id(a, par, npar, i)]);
+        if (staged) skey[i] = k;
+        kmax = max(kmax, k);
+    }
+    kmax = block_max_u32(kmax, sh_u32);
+    const float m = key_to_float(kmax);
+    auto mass = [&](uint32_t k) { return mass_fixed(expf(key_to_float(k) - m)); };
 
     const bool open_all = (a.mode == ZHA_TOP_P && a.p >= 1.f) || (a.mode == ZHA_TOP_K && (long long)a.k >= F);
     uint32_t kstar = 0;
     unsigned long long cstar = 0;
     if (F > 0 && !open_all) {
-        float m = -INFINITY;
-        for (long long i = beg; i < end; ++i) m = fmaxf(m, S[frontier_id(a, par, npar, i)]);
-        m = block_max(m, sh_f);
         unsigned long long trem = 0;
         unsigned krem = (unsigned)a.k;
         if (a.mode == ZHA_TOP_P) {
             unsigned long long z = 0;
-            for (long long i = beg; i < end; ++i) z += mass_fixed(expf(S[frontier_id(a, par, npar, i)] - m));
+            for (long long i = tid; i < F; i += SEL_THREADS) z += mass(key_at(i));
             unsigned long long Z;
             block_incl_scan<unsigned long long>(z, sh_u64, &Z);
             trem = (unsigned long long)ceil((double)a.p * (double)Z);
             if (trem < 1) trem = 1;
             if (trem > Z) trem = Z;
         }
+        // radix select from the top byte down; every bucket carries its count, its
+        // mass and its largest key, so a bucket holding one key ends the search
         uint32_t prefix = 0, pmask = 0;
+        if (tid == 0) s_done = 0;
+        const int copy = (tid >> 5) & (HCOPIES - 1);
         for (int shift = 24; shift >= 0; shift -= 8) {
-            h_mass[tid] = 0;
-            h_cnt[tid] = 0;
+#pragma unroll
+            for (int c = 0; c < HCOPIES; ++c) {
+                h_mass[c][tid] = 0;
+                h_cnt[c][tid] = 0;
+                h_max[c][tid] = 0;
+            }
             __syncthreads();
-            for (long long i = beg; i < end; ++i) {
-                const float s = S[frontier_id(a, par, npar, i)];
-                const uint32_t key = order_key(s);
-                if ((key & pmask) == prefix) {
-                    const int b = (key >> shift) & 255;
-                    atomicAdd(&h_cnt[b], 1u);
-                    if (a.mode == ZHA_TOP_P) atomicAdd(&h_mass[b], mass_fixed(expf(s - m)));
+            for (long long i = tid; i < F; i += SEL_THREADS) {
+                const uint32_t k = key_at(i);
+                if ((k & pmask) == prefix) {
+                    const int b = (k >> shift) & 255;
+                    atomicAdd(&h_cnt[copy][b], 1u);
+                    atomicMax(&h_max[copy][b], k);
+                    if (a.mode == ZHA_TOP_P) atomicAdd(&h_mass[copy][b], mass(k));
                 }
             }
             __syncthreads();
             const int b = 255 - tid;  // thread tid holds the tid-th bucket from the top
-            const unsigned long long vm = h_mass[b];
-            const unsigned vc = h_cnt[b];
+            unsigned long long vm = 0;
+            unsigned vc = 0, vx = 0;
+#pragma unroll
+            for (int c = 0; c < HCOPIES; ++c) {
+                vm += h_mass[c][b];
+                vc += h_cnt[c][b];
+                vx = max(vx, h_max[c][b]);
+            }
             const unsigned long long incl_m = block_incl_scan<unsigned long long>(vm, sh_u64, nullptr);
             const unsigned incl_c = block_incl_scan<unsigned>(vc, sh_u32, nullptr);
             const bool hit = a.mode == ZHA_TOP_P ? (incl_m - vm < trem && trem <= incl_m)
                                                  : (incl_c - vc < krem && krem <= incl_c);
             if (hit) {
-                s_prefix = prefix | ((uint32_t)b << shift);
+                s_prefix = vc == 1 ? vx : (prefix | ((uint32_t)b << shift));
                 s_trem = trem - (incl_m - vm);
                 s_krem = krem - (incl_c - vc);
+                s_done = vc == 1;
             }
             __syncthreads();
             prefix = s_prefix;
             trem = s_trem;
             krem = s_krem;
             pmask |= 255u << shift;
+            const bool done = s_done;
             __syncthreads();
+            if (done) break;
         }
         kstar = prefix;
         if (a.mode == ZHA_TOP_P) {
-            const unsigned long long u = mass_fixed(expf(key_to_float(kstar) - m));
+            const unsigned long long u = mass(kstar);
             cstar = u > 0 ? (trem + u - 1) / u : 1;
         } else {
             cstar = krem;
         }
     }
 
-    // opened = score key above kstar, or equal to it and among the first cstar (by id)
+    // opened = key above kstar, or equal to it and among the first cstar (by id);
+    // each thread owns a contiguous run of positions so that ranks follow ids
+    const long long per = (F + SEL_THREADS - 1) / SEL_THREADS;
+    const long long beg = min(F, tid * per), end = min(F, beg + per);
     unsigned eq_local = 0;
     if (!open_all)
-        for (long long i = beg; i < end; ++i)
-            eq_local += order_key(S[frontier_id(a, par, npar, i)]) == kstar;
+        for (long long i = beg; i < end; ++i) eq_local += key_at(i) == kstar;
     unsigned eq_base = block_incl_scan<unsigned>(eq_local, sh_u32, nullptr) - eq_local;
     unsigned open_local = 0;
     {
@@ -362,7 +403,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_level_kernel(SelectArgs a)
         for (long long i = beg; i < end; ++i) {
             bool o = open_all;
             if (!open_all) {
-                const uint32_t key = order_key(S[frontier_id(a, par, npar, i)]);
+                const uint32_t key = key_at(i);
                 o = key > kstar || (key == kstar && eq < cstar);
                 eq += key == kstar;
             }
@@ -378,14 +419,14 @@ __global__ void __launch_bounds__(SEL_THREADS) select_level_kernel(SelectArgs a)
         unsigned *M_tree = a.M_next ? a.M_next + (long long)t * a.words_next * a.G : nullptr;
         unsigned *U_tree = a.U_next ? a.U_next + (long long)t * a.words_next : nullptr;
         for (long long i = beg; i < end; ++i) {
-            const long long id = frontier_id(a, par, npar, i);
             bool o = open_all;
             if (!open_all) {
-                const uint32_t key = order_key(S[id]);
+                const uint32_t key = key_at(i);
                 o = key > kstar || (key == kstar && eq < cstar);
                 eq += key == kstar;
             }
             if (!o) continue;
+            const long long id = frontier_id(a, par, npar, i);
             if (a.level == 1) {
                 if (rank < (unsigned)a.max_sel) a.sel[walk * a.max_sel + rank] = (int)id;
             } else {
@@ -461,7 +502,7 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
     }
     auto words = [&](int l) { return (t->cap_nodes[l] + 31) / 32; };
 
-    InitArgs ia;
+    InitArgs ia{};
     ia.Q = Q;
     ia.q_bf16 = q_dtype == ZHA_BF16;
     ia.D = D;
@@ -483,7 +524,7 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
 
     int cur = 0;
     for (int l = start_level; l >= 1; --l) {
-        ScoreArgs sa;
+        ScoreArgs sa{};
         sa.nodes = t->nodes[l];
         sa.node_tree = t->cap_nodes[l] * t->NF;
         sa.NF = t->NF;
@@ -505,7 +546,7 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
         }
         if (e != cudaSuccess) return e;
 
-        SelectArgs se;
+        SelectArgs se{};
         se.level = l;
         se.C = C;
         se.R = c.R;
@@ -534,9 +575,17 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
         se.stats = stats;
         se.tail = t->n - (long long)C * t->n_nodes[1];
         se.status = t->d_status;
+        se.smem_keys = std::min<long long>(t->n_nodes[l], SEL_SMEM_KEYS);
+        static bool smem_set = false;
+        if (!smem_set) {
+            e = cudaFuncSetAttribute(select_level_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     SEL_SMEM_KEYS * (int)sizeof(uint32_t));
+            if (e != cudaSuccess) return e;
+            smem_set = true;
+        }
         {
             Probe pr(t, ZHA_K_SELECT, st);
-            select_level_kernel<<<(unsigned)W, SEL_THREADS, 0, st>>>(se);
+            select_level_kernel<<<(unsigned)W, SEL_THREADS, (size_t)se.smem_keys * sizeof(uint32_t), st>>>(se);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
         cur ^= 1;
