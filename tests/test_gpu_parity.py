@@ -280,6 +280,17 @@ def test_odd_reference_count_and_chunk():
     _check_against_oracle(K, V, refs, Q, 2000, 5, 4, 0.2, modes=ALL_MODES)
 
 
+def test_large_frontiers():
+    # 200,000 keys, C = 8: 25,000 level-1 nodes under 3,125 level-2 nodes; with the
+    # walk starting at level 2, the level-1 frontier reaches 25,000 nodes (more
+    # than a 512-thread selector stages in shared memory) at p = 1, and between
+    # 8,192 and 16,384 nodes for the smaller p
+    K, V, refs, Q = _tiny(200000, C=8, depth=2, d=64, R=2, nq=3, seed=5)
+    _check_against_oracle(K, V, refs, Q, 200000, 8, 2, 0.125, top_width=4096,
+                          modes=((O.TOP_P, 1.0, 0), (O.TOP_P, 0.9, 0), (O.TOP_P, 0.5, 0), (O.TOP_K, 0, 2500),
+                                 (O.TOP_K, 0, 1500)))
+
+
 def test_max_sel_overflow_is_reported():
     Z = zha()
     K, V, refs, Q = _tiny(1024, C=8, depth=2)

@@ -158,6 +158,7 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     };
     const size_t o_qf = take(sizeof(float) * W * c.d);
     const size_t o_S = take(sizeof(float) * W * cap1);
+    const size_t o_gk = take(sizeof(uint32_t) * W * cap1);
     const size_t o_L0 = take(sizeof(int) * W * cap2);
     const size_t o_L1 = take(sizeof(int) * W * cap2);
     const size_t o_c0 = take(sizeof(int) * W);
@@ -172,6 +173,7 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     const size_t U_bytes = off - U_start;
     const size_t o_io = take(sizeof(int) * (W + 1));
     const size_t o_iw = take(sizeof(int) * max_items);
+    const size_t o_wd = take(sizeof(int) * W);
     const size_t o_pa = take(sizeof(float) * max_items * (c.d + 2));
     const size_t need = off;
 
@@ -189,6 +191,7 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     char *b = static_cast<char *>(t->ws);
     s->qf = reinterpret_cast<float *>(b + o_qf);
     s->S = reinterpret_cast<float *>(b + o_S);
+    s->gkey = reinterpret_cast<uint32_t *>(b + o_gk);
     s->L[0] = reinterpret_cast<int *>(b + o_L0);
     s->L[1] = reinterpret_cast<int *>(b + o_L1);
     s->cnt[0] = reinterpret_cast<int *>(b + o_c0);
@@ -203,6 +206,7 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     s->U_bytes = U_bytes;
     s->item_off = reinterpret_cast<int *>(b + o_io);
     s->item_walk = reinterpret_cast<int *>(b + o_iw);
+    s->walk_done = reinterpret_cast<int *>(b + o_wd);
     s->partial = reinterpret_cast<float *>(b + o_pa);
     s->Sstride = cap1;
     s->Lstride = cap2;

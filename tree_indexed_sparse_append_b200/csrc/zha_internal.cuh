@@ -193,6 +193,7 @@ namespace zha {
 struct Scratch {
     float *qf;                 // [W][D] queries as fp32
     float *S;                  // [W][Sstride] node scores, indexed by node id
+    uint32_t *gkey;            // [W][Sstride] frontier keys too many for shared memory
     int *L[2];                 // [W][Lstride] frontier lists (ping-pong)
     int *cnt[2];               // [W] frontier counts
     unsigned *M[ZHA_MAX_DEPTH + 1];  // per level: [T][words_l][G] membership bits
@@ -201,6 +202,7 @@ struct Scratch {
     unsigned *M_base, *U_base;
     int *item_off;             // [W + 1] attend items per walk (prefix)
     int *item_walk;            // [max_items] walk of each attend item
+    int *walk_done;            // [W] attend items finished per walk
     float *partial;            // [max_items][D + 2]
     long long Sstride, Lstride, max_items;
 };

@@ -39,10 +39,9 @@
 namespace zha {
 namespace {
 
-constexpr int SEL_THREADS = 256;
 
 // ---------------------------------------------------------------------------
-// block-wide helpers for SEL_THREADS threads (8 warps)
+// block-wide helpers
 template <typename V>
 __device__ __forceinline__ V warp_incl_scan(V x, int lane) {
 #pragma unroll
@@ -53,21 +52,21 @@ __device__ __forceinline__ V warp_incl_scan(V x, int lane) {
     return x;
 }
 
-// inclusive scan across the block; `sh` holds 8 + 1 values
-template <typename V>
+// inclusive scan across a block of NT threads; `sh` holds NT / 32 values
+template <int NT, typename V>
 __device__ __forceinline__ V block_incl_scan(V x, V *sh, V *total) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     V inc = warp_incl_scan(x, lane);
     if (lane == 31) sh[w] = inc;
     __syncthreads();
     if (w == 0) {
-        V s = lane < SEL_THREADS / 32 ? sh[lane] : V(0);
+        V s = lane < NT / 32 ? sh[lane] : V(0);
         s = warp_incl_scan(s, lane);
-        if (lane < SEL_THREADS / 32) sh[lane] = s;
+        if (lane < NT / 32) sh[lane] = s;
     }
     __syncthreads();
     V base = w > 0 ? sh[w - 1] : V(0);
-    if (total) *total = sh[SEL_THREADS / 32 - 1];
+    if (total) *total = sh[NT / 32 - 1];
     __syncthreads();
     return base + inc;
 }
@@ -224,6 +223,7 @@ __global__ void __launch_bounds__(256) score_level_kernel(ScoreArgs a) {
 // ---------------------------------------------------------------------------
 struct SelectArgs {
     int level, C, R, G;
+    int c_shift;             // log2(C) when C is a power of two, else -1
     int start;               // 1 when this level is the start level (frontier = all nodes)
     long long n_level;       // nodes at this level
     long long n_orph;        // orphans at this level (nodes past C * n_{level+1}); 0 at start
@@ -248,17 +248,23 @@ struct SelectArgs {
     long long tail;
     int *status;
     long long smem_keys;     // frontiers up to this size are staged in shared memory
+    uint32_t *gkey;          // [W][Sstride] staging for larger frontiers
 };
 
-// frontier position -> node id
+// frontier position -> node id (positions and ids fit in 32 bits)
 __device__ __forceinline__ long long frontier_id(const SelectArgs &a, const int *par, long long npar,
                                                  long long i) {
     if (a.start) return i;
-    const long long kids = npar * a.C;
-    if (i < kids) return (long long)par[i / a.C] * a.C + i % a.C;
-    return (a.n_level - a.n_orph) + (i - kids);
+    const int ii = (int)i, C = a.C;
+    const int kids = (int)npar * C;
+    if (ii < kids) {
+        const int pi = a.c_shift >= 0 ? ii >> a.c_shift : ii / C;
+        return (long long)par[pi] * C + (ii - pi * C);
+    }
+    return (a.n_level - a.n_orph) + (ii - kids);
 }
 
+template <int NT>
 __device__ __forceinline__ uint32_t block_max_u32(uint32_t x, unsigned *sh) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
 #pragma unroll
@@ -267,29 +273,48 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t x, unsigned *sh) {
     __syncthreads();
     uint32_t r = sh[0];
 #pragma unroll
-    for (int i = 1; i < SEL_THREADS / 32; ++i) r = max(r, sh[i]);
+    for (int i = 1; i < NT / 32; ++i) r = max(r, sh[i]);
     __syncthreads();
     return r;
 }
 
-// Each walk's frontier keys are staged once in shared memory (up to
-// SEL_SMEM_KEYS of them; larger frontiers are re-read from the score array).
-// Histograms are kept in HCOPIES copies (warp w uses copy w % HCOPIES) so that
-// lanes with equal top bits contend less.
-constexpr int SEL_SMEM_KEYS = 8192;
-constexpr int HCOPIES = 4;
+// Each walk's frontier keys are staged once, in shared memory when they fit
+// (smem_keys), else in the walk's row of a global key array. The cutoff is found
+// with at most three kinds of histogram pass, each over 256 buckets that keep
+// count, fixed-point mass and largest key (HCOPIES copies, shared by groups of
+// warps):
+//   1. coarse: 1/8 nat per bucket below the frontier's highest score (keys
+//      spread over many buckets, so the atomics rarely collide; this pass also
+//      yields the total mass);
+//   2. fine: 1/2048 nat inside the crossing coarse bucket;
+//   3. radix on the raw score bits inside the crossing fine bucket, a byte at a
+//      time (only when several keys share that 1/2048-nat bucket).
+// Bucket orders agree with the score order, so the crossing bucket of each pass
+// holds the cutoff; a bucket with a single key ends the search.
+constexpr int HCOPIES = 8;
+constexpr float COARSE_PER_NAT = 8.f;
 
-__global__ void __launch_bounds__(SEL_THREADS) select_level_kernel(SelectArgs a) {
-    extern __shared__ uint32_t skey[];
+__device__ __forceinline__ int coarse_bucket(float s, float m) {
+    const float x = (m - s) * COARSE_PER_NAT;
+    return x >= 255.f ? 255 : (x > 0.f ? (int)x : 0);
+}
+__device__ __forceinline__ int fine_bucket(float s, float m, int cb) {
+    const float y = ((m - s) * COARSE_PER_NAT - (float)cb) * 256.f;
+    return y >= 255.f ? 255 : (y > 0.f ? (int)y : 0);
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
+    extern __shared__ uint32_t skey_s[];
     __shared__ unsigned long long h_mass[HCOPIES][256];
     __shared__ unsigned h_cnt[HCOPIES][256];
     __shared__ unsigned h_max[HCOPIES][256];
-    __shared__ unsigned long long sh_u64[SEL_THREADS / 32];
-    __shared__ unsigned sh_u32[SEL_THREADS / 32];
-    __shared__ uint32_t s_prefix;
+    __shared__ unsigned long long sh_u64[NT / 32];
+    __shared__ unsigned sh_u32[NT / 32];
+    __shared__ int s_bucket;
+    __shared__ uint32_t s_key;
     __shared__ unsigned long long s_trem;
-    __shared__ unsigned s_krem;
-    __shared__ int s_done;
+    __shared__ unsigned s_krem, s_count;
 
     const long long walk = blockIdx.x;
     const int tid = threadIdx.x;
@@ -298,91 +323,134 @@ __global__ void __launch_bounds__(SEL_THREADS) select_level_kernel(SelectArgs a)
     const int *par = a.par_in + walk * a.Lstride;
     const long long F = a.start ? a.n_level : npar * a.C + a.n_orph;
     const float *S = a.S + walk * a.Sstride;
-    const bool staged = F <= a.smem_keys;
-    auto key_at = [&](long long i) -> uint32_t {
-        return staged ? skey[i] : order_key(S[frontier_id(a, par, npar, i)]);
-    };
+    uint32_t *skey = F <= a.smem_keys ? skey_s : a.gkey + walk * a.Sstride;
+    auto key_at = [&](long long i) -> uint32_t { return skey[i]; };
 
     // stage the frontier's keys (coalesced, strided) and find the largest
     uint32_t kmax = 0;
-    for (long long i = tid; i < F; i += SEL_THREADS) {
-        const uint32_t k = order_key(S[frontier_id(a, par, npar, i)]);
-        if (staged) skey[i] = k;
-        kmax = max(kmax, k);
+    {
+        long long i = tid;
+        for (; i + 7 * NT < F; i += 8 * NT) {
+            long long id[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) id[u] = frontier_id(a, par, npar, i + u * NT);
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = S[id[u]];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t k = order_key(v[u]);
+                skey[i + u * NT] = k;
+                kmax = max(kmax, k);
+            }
+        }
+        for (; i < F; i += NT) {
+            const uint32_t k = order_key(S[frontier_id(a, par, npar, i)]);
+            skey[i] = k;
+            kmax = max(kmax, k);
+        }
     }
-    kmax = block_max_u32(kmax, sh_u32);
+    kmax = block_max_u32<NT>(kmax, sh_u32);
     const float m = key_to_float(kmax);
-    auto mass = [&](uint32_t k) { return mass_fixed(expf(key_to_float(k) - m)); };
+    auto mass = [&](float s) { return mass_fixed(expf(s - m)); };
 
     const bool open_all = (a.mode == ZHA_TOP_P && a.p >= 1.f) || (a.mode == ZHA_TOP_K && (long long)a.k >= F);
+    const bool top_p = a.mode == ZHA_TOP_P;
     uint32_t kstar = 0;
     unsigned long long cstar = 0;
+    unsigned eq_count = 0;  // keys equal to kstar
     if (F > 0 && !open_all) {
         unsigned long long trem = 0;
         unsigned krem = (unsigned)a.k;
-        if (a.mode == ZHA_TOP_P) {
-            unsigned long long z = 0;
-            for (long long i = tid; i < F; i += SEL_THREADS) z += mass(key_at(i));
-            unsigned long long Z;
-            block_incl_scan<unsigned long long>(z, sh_u64, &Z);
-            trem = (unsigned long long)ceil((double)a.p * (double)Z);
-            if (trem < 1) trem = 1;
-            if (trem > Z) trem = Z;
-        }
-        // radix select from the top byte down; every bucket carries its count, its
-        // mass and its largest key, so a bucket holding one key ends the search
+        const int wcopy = (tid >> 5) & (HCOPIES - 1);
+        // stage 0: coarse, 1: fine, 2..5: raw bytes 24, 16, 8, 0
+        int cb = -1, fb = -1;
         uint32_t prefix = 0, pmask = 0;
-        if (tid == 0) s_done = 0;
-        const int copy = (tid >> 5) & (HCOPIES - 1);
-        for (int shift = 24; shift >= 0; shift -= 8) {
-#pragma unroll
-            for (int c = 0; c < HCOPIES; ++c) {
-                h_mass[c][tid] = 0;
-                h_cnt[c][tid] = 0;
-                h_max[c][tid] = 0;
+        bool done = false;
+        for (int stage = 0; stage < 6 && !done; ++stage) {
+            for (int j = tid; j < HCOPIES * 256; j += NT) {
+                (&h_mass[0][0])[j] = 0;
+                (&h_cnt[0][0])[j] = 0;
+                (&h_max[0][0])[j] = 0;
             }
             __syncthreads();
-            for (long long i = tid; i < F; i += SEL_THREADS) {
+            const int shift = 24 - 8 * (stage - 2);
+            for (long long i = tid; i < F; i += NT) {
                 const uint32_t k = key_at(i);
-                if ((k & pmask) == prefix) {
-                    const int b = (k >> shift) & 255;
-                    atomicAdd(&h_cnt[copy][b], 1u);
-                    atomicMax(&h_max[copy][b], k);
-                    if (a.mode == ZHA_TOP_P) atomicAdd(&h_mass[copy][b], mass(k));
+                const float s = key_to_float(k);
+                int b;
+                if (stage == 0) {
+                    b = coarse_bucket(s, m);
+                } else {
+                    if (coarse_bucket(s, m) != cb) continue;
+                    if (stage == 1) {
+                        b = fine_bucket(s, m, cb);
+                    } else {
+                        if (fine_bucket(s, m, cb) != fb || (k & pmask) != prefix) continue;
+                        b = (k >> shift) & 255;
+                    }
+                }
+                atomicAdd(&h_cnt[wcopy][b], 1u);
+                atomicMax(&h_max[wcopy][b], k);
+                if (top_p) atomicAdd(&h_mass[wcopy][b], mass(s));
+            }
+            __syncthreads();
+            // threads 0..255 own one bucket each: buckets ascend from the highest
+            // scores (stages 0, 1) or descend (raw bytes), so raw stages read them
+            // in reverse; threads past 255 add nothing to the scans
+            const bool own = tid < 256;
+            const int b = own ? (stage >= 2 ? 255 - tid : tid) : 0;
+            unsigned long long vm = 0;
+            unsigned vc = 0, vx = 0;
+            if (own) {
+#pragma unroll
+                for (int c = 0; c < HCOPIES; ++c) {
+                    vm += h_mass[c][b];
+                    vc += h_cnt[c][b];
+                    vx = max(vx, h_max[c][b]);
+                }
+            }
+            unsigned long long total_m;
+            const unsigned long long incl_m = block_incl_scan<NT, unsigned long long>(vm, sh_u64, &total_m);
+            const unsigned incl_c = block_incl_scan<NT, unsigned>(vc, sh_u32, nullptr);
+            if (stage == 0 && top_p) {
+                trem = (unsigned long long)ceil((double)a.p * (double)total_m);
+                if (trem < 1) trem = 1;
+                if (trem > total_m) trem = total_m;
+            }
+            const bool hit = own && (top_p ? (incl_m - vm < trem && trem <= incl_m)
+                                           : (incl_c - vc < krem && krem <= incl_c));
+            if (hit) {
+                s_bucket = b;
+                s_key = vx;
+                s_trem = trem - (incl_m - vm);
+                s_krem = krem - (incl_c - vc);
+                s_count = vc;
+            }
+            __syncthreads();
+            const int hb = s_bucket;
+            trem = s_trem;
+            krem = s_krem;
+            eq_count = s_count;
+            if (eq_count == 1) {
+                kstar = s_key;
+                done = true;
+            } else if (stage == 0) {
+                cb = hb;
+            } else if (stage == 1) {
+                fb = hb;
+            } else {
+                prefix |= (uint32_t)hb << shift;
+                pmask |= 255u << shift;
+                if (stage == 5) {
+                    kstar = prefix;
+                    done = true;
                 }
             }
             __syncthreads();
-            const int b = 255 - tid;  // thread tid holds the tid-th bucket from the top
-            unsigned long long vm = 0;
-            unsigned vc = 0, vx = 0;
-#pragma unroll
-            for (int c = 0; c < HCOPIES; ++c) {
-                vm += h_mass[c][b];
-                vc += h_cnt[c][b];
-                vx = max(vx, h_max[c][b]);
-            }
-            const unsigned long long incl_m = block_incl_scan<unsigned long long>(vm, sh_u64, nullptr);
-            const unsigned incl_c = block_incl_scan<unsigned>(vc, sh_u32, nullptr);
-            const bool hit = a.mode == ZHA_TOP_P ? (incl_m - vm < trem && trem <= incl_m)
-                                                 : (incl_c - vc < krem && krem <= incl_c);
-            if (hit) {
-                s_prefix = vc == 1 ? vx : (prefix | ((uint32_t)b << shift));
-                s_trem = trem - (incl_m - vm);
-                s_krem = krem - (incl_c - vc);
-                s_done = vc == 1;
-            }
-            __syncthreads();
-            prefix = s_prefix;
-            trem = s_trem;
-            krem = s_krem;
-            pmask |= 255u << shift;
-            const bool done = s_done;
-            __syncthreads();
-            if (done) break;
         }
-        kstar = prefix;
-        if (a.mode == ZHA_TOP_P) {
-            const unsigned long long u = mass(kstar);
+        if (top_p) {
+            const unsigned long long u = mass(key_to_float(kstar));
             cstar = u > 0 ? (trem + u - 1) / u : 1;
         } else {
             cstar = krem;
@@ -391,12 +459,14 @@ __global__ void __launch_bounds__(SEL_THREADS) select_level_kernel(SelectArgs a)
 
     // opened = key above kstar, or equal to it and among the first cstar (by id);
     // each thread owns a contiguous run of positions so that ranks follow ids
-    const long long per = (F + SEL_THREADS - 1) / SEL_THREADS;
+    const long long per = (F + NT - 1) / NT;
     const long long beg = min(F, tid * per), end = min(F, beg + per);
+    // ranks among keys equal to kstar matter only when some of them stay closed
+    const bool split_tie = !open_all && cstar < eq_count;
     unsigned eq_local = 0;
-    if (!open_all)
+    if (split_tie)
         for (long long i = beg; i < end; ++i) eq_local += key_at(i) == kstar;
-    unsigned eq_base = block_incl_scan<unsigned>(eq_local, sh_u32, nullptr) - eq_local;
+    unsigned eq_base = split_tie ? block_incl_scan<NT, unsigned>(eq_local, sh_u32, nullptr) - eq_local : 0u;
     unsigned open_local = 0;
     {
         unsigned eq = eq_base;
@@ -411,7 +481,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_level_kernel(SelectArgs a)
         }
     }
     unsigned n_open;
-    unsigned open_base = block_incl_scan<unsigned>(open_local, sh_u32, &n_open) - open_local;
+    unsigned open_base = block_incl_scan<NT, unsigned>(open_local, sh_u32, &n_open) - open_local;
 
     // write the opened ids (ascending, since frontier positions ascend in id)
     {
@@ -437,7 +507,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_level_kernel(SelectArgs a)
         }
         if (a.level > 1 && a.n_orph_next > 0) {
             const long long lo = a.n_level_next - a.n_orph_next, hi = a.n_level_next;
-            for (long long w = (lo >> 5) + tid; w <= (hi - 1) >> 5; w += SEL_THREADS) {
+            for (long long w = (lo >> 5) + tid; w <= (hi - 1) >> 5; w += NT) {
                 const long long wlo = lo > (w << 5) ? lo : (w << 5);
                 const long long whi = hi < ((w + 1) << 5) ? hi : ((w + 1) << 5);
                 set_bits(M_tree, U_tree, a.G, g, wlo, whi);
@@ -463,6 +533,19 @@ __global__ void __launch_bounds__(SEL_THREADS) select_level_kernel(SelectArgs a)
             }
         }
     }
+}
+
+template <int NT>
+cudaError_t launch_select(const SelectArgs &se, long long W, cudaStream_t st) {
+    static bool smem_set = false;
+    if (!smem_set) {
+        cudaError_t e = cudaFuncSetAttribute(select_level_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             16384 * (int)sizeof(uint32_t));
+        if (e != cudaSuccess) return e;
+        smem_set = true;
+    }
+    select_level_kernel<NT><<<(unsigned)W, NT, (size_t)se.smem_keys * sizeof(uint32_t), st>>>(se);
+    return cudaGetLastError();
 }
 
 template <int D, int RP>
@@ -549,6 +632,7 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
         SelectArgs se{};
         se.level = l;
         se.C = C;
+        se.c_shift = (C & (C - 1)) == 0 ? __builtin_ctz((unsigned)C) : -1;
         se.R = c.R;
         se.G = G;
         se.start = l == start_level;
@@ -575,18 +659,17 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
         se.stats = stats;
         se.tail = t->n - (long long)C * t->n_nodes[1];
         se.status = t->d_status;
-        se.smem_keys = std::min<long long>(t->n_nodes[l], SEL_SMEM_KEYS);
-        static bool smem_set = false;
-        if (!smem_set) {
-            e = cudaFuncSetAttribute(select_level_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     SEL_SMEM_KEYS * (int)sizeof(uint32_t));
-            if (e != cudaSuccess) return e;
-            smem_set = true;
-        }
+        se.gkey = s.gkey;
         {
             Probe pr(t, ZHA_K_SELECT, st);
-            select_level_kernel<<<(unsigned)W, SEL_THREADS, (size_t)se.smem_keys * sizeof(uint32_t), st>>>(se);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            if (t->n_nodes[l] > 8192) {
+                se.smem_keys = std::min<long long>(t->n_nodes[l], 16384);
+                e = launch_select<512>(se, W, st);
+            } else {
+                se.smem_keys = t->n_nodes[l];
+                e = launch_select<256>(se, W, st);
+            }
+            if (e != cudaSuccess) return e;
         }
         cur ^= 1;
     }
