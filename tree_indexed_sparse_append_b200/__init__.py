@@ -29,7 +29,7 @@ SYMBOLS = ("zha_build", "zha_append", "zha_search", "zha_attend", "zha_reserve",
            "zha_num_keys", "zha_sync_status", "zha_destroy", "zha_last_error", "zha_version",
            "zha_profile", "zha_profile_read", "zha_kernel_launches", "zha_last_search_info")
 KERNEL_KINDS = ("build", "append", "search_init", "score", "select", "attend_plan", "attend_partial",
-                "attend_combine")
+                "attend_combine", "union")
 
 
 class ZhaError(RuntimeError):

@@ -142,10 +142,10 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     (void)G;
     const long long cap1 = t->cap_nodes[1] > 0 ? t->cap_nodes[1] : 1;
     const long long cap2 = c.depth >= 2 && t->cap_nodes[2] > 0 ? t->cap_nodes[2] : 1;
-    // attend items: a walk's keys (at most C * (max_sel + 1)) in items of >= 64 keys,
+    // attend items: a walk's keys (at most C * (max_sel + 1)) in items of >= 128 keys,
     // at most 128 items per walk (constants of zha_attend.cu)
     const long long keys_max = (long long)c.chunk * ((long long)max_sel + 1);
-    long long per_walk_items = (keys_max + 63) / 64;
+    long long per_walk_items = (keys_max + 127) / 128;
     if (per_walk_items > 128) per_walk_items = 128;
     if (per_walk_items < 1) per_walk_items = 1;
     const long long max_items = W * per_walk_items;

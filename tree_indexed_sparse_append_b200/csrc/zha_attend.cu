@@ -31,7 +31,7 @@
 namespace zha {
 namespace {
 
-constexpr int SEG = 64;         // keys per work item, at least
+constexpr int SEG = 128;        // keys per work item, at least
 constexpr int MAX_SPLIT = 128;  // work items per walk, at most
 
 __device__ __forceinline__ long long walk_keys(const int *sel_count, long long w, int max_sel, int C,

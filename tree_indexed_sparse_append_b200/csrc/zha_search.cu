@@ -155,66 +155,101 @@ struct ScoreArgs {
     const float *qf;
     float *S;
     long long Sstride;
+    int npi;  // node ids per work item: 4, or 1 for small levels
 };
 
 template <int D, int RP>
-__global__ void __launch_bounds__(256) score_level_kernel(ScoreArgs a) {
+__device__ __forceinline__ void load_node(const float *node, int R, int lane, float (&kr)[RP][D / 32]) {
+    constexpr int EPL = D / 32;
+#pragma unroll
+    for (int r = 0; r < RP; ++r) {
+        if (r < R) {
+            load_f32<EPL>(node + r * D + lane * EPL, kr[r]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) kr[r][e] = 0.f;
+        }
+    }
+}
+
+// Scores one node (rows in kr) against every walk of tree t whose frontier
+// holds node j.
+template <int D, int RP>
+__device__ __forceinline__ void score_node(const ScoreArgs &a, int t, long long j, const float (&kr)[RP][D / 32],
+                                           float bias, int lane) {
     constexpr int EPL = D / 32;
     constexpr int LG = ilog2(RP);
-    const int lane = threadIdx.x & 31;
     const int rr = lane >> (5 - LG);  // row whose full dot product this lane ends with
-    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
-    const long long groups = (a.n_level + 3) >> 2;
-    const long long items = groups * a.T;
-
-    for (long long it = gw; it < items; it += nw) {
-        const int t = (int)(it / groups);
-        const long long j0 = (it - (long long)t * groups) << 2;
-        const unsigned word = a.U[(long long)t * a.words + (j0 >> 5)];
-        unsigned nib = (word >> (j0 & 31)) & 0xFu;
-        while (nib) {
-            const int b = __ffs(nib) - 1;
-            nib &= nib - 1;
-            const long long j = j0 + b;
-            const float *node = a.nodes + (long long)t * a.node_tree + j * a.NF;
-            float kr[RP][EPL];
+    const unsigned *Mrow = a.M + ((long long)t * a.words + (j >> 5)) * a.G;
+    const int bit = (int)(j & 31);
+    for (int g0 = 0; g0 < a.G; g0 += 32) {
+        const unsigned mw = (g0 + lane < a.G) ? __ldg(Mrow + g0 + lane) : 0u;
+        unsigned members = __ballot_sync(FULL, (mw >> bit) & 1u);
+        while (members) {
+            const int gl = __ffs(members) - 1;
+            members &= members - 1;
+            const long long walk = (long long)t * a.G + g0 + gl;
+            float q[EPL];
+            load_q<EPL>(a.qf + walk * D + lane * EPL, q);
+            float part[RP];
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
-                if (r < a.R) {
-                    load_f32<EPL>(node + r * D + lane * EPL, kr[r]);
-                } else {
+                float s = 0.f;
 #pragma unroll
-                    for (int e = 0; e < EPL; ++e) kr[r][e] = 0.f;
-                }
+                for (int e = 0; e < EPL; ++e) s = fmaf(kr[r][e], q[e], s);
+                part[r] = s;
             }
-            const float bias = rr < a.R ? __ldg(node + a.R * D + rr) : 0.f;
-            const unsigned *Mrow = a.M + ((long long)t * a.words + (j >> 5)) * a.G;
-            const int bit = (int)(j & 31);
-            for (int g0 = 0; g0 < a.G; g0 += 32) {
-                const unsigned mw = (g0 + lane < a.G) ? __ldg(Mrow + g0 + lane) : 0u;
-                unsigned members = __ballot_sync(FULL, (mw >> bit) & 1u);
-                while (members) {
-                    const int gl = __ffs(members) - 1;
-                    members &= members - 1;
-                    const long long walk = (long long)t * a.G + g0 + gl;
-                    float q[EPL];
-                    load_q<EPL>(a.qf + walk * D + lane * EPL, q);
-                    float part[RP];
+            const float dot = transpose_reduce<RP>(part, lane);
+            float sc = rr < a.R ? fmaf(a.beta, dot, bias) : -INFINITY;
 #pragma unroll
-                    for (int r = 0; r < RP; ++r) {
-                        float s = 0.f;
-#pragma unroll
-                        for (int e = 0; e < EPL; ++e) s = fmaf(kr[r][e], q[e], s);
-                        part[r] = s;
-                    }
-                    const float dot = transpose_reduce<RP>(part, lane);
-                    float sc = rr < a.R ? fmaf(a.beta, dot, bias) : -INFINITY;
-#pragma unroll
-                    for (int off = 16; off >= (32 >> LG) && LG > 0; off >>= 1)
-                        sc = fmaxf(sc, __shfl_xor_sync(FULL, sc, off));
-                    if (lane == 0) a.S[walk * a.Sstride + j] = sc;
-                }
+            for (int off = 16; off >= (32 >> LG) && LG > 0; off >>= 1) sc = fmaxf(sc, __shfl_xor_sync(FULL, sc, off));
+            if (lane == 0) a.S[walk * a.Sstride + j] = sc;
+        }
+    }
+}
+
+// Grid-stride over (tree, group of npi node ids) items of the level's union
+// bitmap (npi = 4, or 1 for levels too small to give every warp several items).
+// Each lane fetches the union bits of one of the warp's next 32 items in a single
+// load, so walking the items costs no memory round trip of its own; every set
+// node is then loaded (R rows of 16-byte lanes) and scored.
+template <int D, int RP>
+__global__ void __launch_bounds__(256, 3) score_level_kernel(ScoreArgs a) {
+    constexpr int LG = ilog2(RP);
+    const int lane = threadIdx.x & 31;
+    const int rr = lane >> (5 - LG);
+    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+    const int npi = a.npi;
+    const unsigned nmask = (1u << npi) - 1u;
+    const long long groups = (a.n_level + npi - 1) / npi;
+    const long long items = groups * a.T;
+
+    for (long long base = gw; base < items; base += 32 * nw) {
+        const long long mine = base + (long long)lane * nw;
+        unsigned my_bits = 0;
+        if (mine < items) {
+            const int t = (int)(mine / groups);
+            const long long j0 = (mine - (long long)t * groups) * npi;
+            my_bits = (__ldg(a.U + (long long)t * a.words + (j0 >> 5)) >> (j0 & 31)) & nmask;
+        }
+        unsigned any = __ballot_sync(FULL, my_bits != 0);
+        while (any) {
+            const int li = __ffs(any) - 1;
+            any &= any - 1;
+            unsigned bits = __shfl_sync(FULL, my_bits, li);
+            const long long it = base + (long long)li * nw;
+            const int t = (int)(it / groups);
+            const long long j0 = (it - (long long)t * groups) * npi;
+            const float *tree_nodes = a.nodes + (long long)t * a.node_tree;
+            while (bits) {
+                const long long j = j0 + __ffs(bits) - 1;
+                bits &= bits - 1;
+                const float *node = tree_nodes + j * a.NF;
+                float kr[RP][D / 32];
+                load_node<D, RP>(node, a.R, lane, kr);
+                const float bias = rr < a.R ? __ldg(node + a.R * D + rr) : 0.f;
+                score_node<D, RP>(a, t, j, kr, bias, lane);
             }
         }
     }
@@ -549,10 +584,18 @@ cudaError_t launch_select(const SelectArgs &se, long long W, cudaStream_t st) {
 }
 
 template <int D, int RP>
-cudaError_t launch_score(const zha_tree *t, const ScoreArgs &a, cudaStream_t st) {
-    const long long items = ((a.n_level + 3) >> 2) * a.T;
+cudaError_t launch_score(const zha_tree *t, ScoreArgs a, cudaStream_t st) {
+    static int per_sm = 0;
+    if (!per_sm) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, score_level_kernel<D, RP>, 256, 0) != cudaSuccess ||
+            per_sm < 1)
+            per_sm = 1;
+    }
+    const long long resident_warps = (long long)num_sms() * per_sm * 8;
+    if (a.T * ((a.n_level + 3) / 4) < 4 * resident_warps) a.npi = 1;
+    const long long items = (long long)a.T * ((a.n_level + a.npi - 1) / a.npi);
     long long blocks = (items + 7) / 8;
-    const long long cap = (long long)num_sms() * 8;
+    const long long cap = (long long)num_sms() * per_sm;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) return cudaSuccess;
     Probe pr(t, ZHA_K_SCORE, st);
@@ -622,6 +665,7 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
         sa.qf = s.qf;
         sa.S = s.S;
         sa.Sstride = s.Sstride;
+        sa.npi = 4;
         switch (D) {
             case 64: e = launch_score_d<64>(t, sa, st); break;
             case 128: e = launch_score_d<128>(t, sa, st); break;
