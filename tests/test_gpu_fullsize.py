@@ -1,0 +1,157 @@
+"""Parity at the workloads' full sizes, in the launch configuration bench.py
+times, on sampled outputs the oracle computes one tree or one walk at a time.
+
+  * 256K keys: 16 sequences x 4 KV heads x 262,144 keys, 256 walks (top-p 0.9);
+    every level of two sampled trees, the walks of those trees, their attention;
+    then 4,096 appends one key at a time through zha_append, the grown nodes and
+    a second search against the oracle's appended trees.
+  * 1M keys: 8 x 8 KV heads x 1,048,576 keys, 256 walks, top-p 0.9 and top-K 16;
+    two sampled trees.
+  * prefill: 4,096 queries x 16 query heads against the 256K trees of sequence 0
+    (65,536 walks); 64 sampled walks.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synthetic as S
+from helpers import (assert_attention_close, assert_nodes_close, compare_selection, gpu_level, host64,
+                     oracle_tree)
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+THREADS = os.cpu_count() or 8
+MODE = {"top_p": O.TOP_P, "top_k": O.TOP_K}
+
+
+def zha():
+    import tree_indexed_sparse_append_b200 as Z
+
+    return Z
+
+
+def walks_of_tree(w, b, h):
+    group = w.n_q_heads // w.n_kv_heads
+    for hq in range(h * group, (h + 1) * group):
+        for i in range(w.queries_per_head):
+            yield (b * w.n_q_heads + hq) * w.queries_per_head + i, hq, i
+
+
+def check_trees(w, inp, tree, sample, n_keys=None, otrees=None):
+    otrees = otrees or {}
+    for b, h in sample:
+        if (b, h) not in otrees:
+            otrees[(b, h)] = oracle_tree(inp, b, h, n_keys=n_keys, threads=THREADS, capacity=w.capacity)
+        ot = otrees[(b, h)]
+        t = b * w.n_kv_heads + h
+        for l in range(1, w.depth + 1):
+            g, n = gpu_level(tree, l, t)
+            assert n == ot.n_nodes[l]
+            if n:
+                assert_nodes_close(g, *ot.level(l), w.R, w.d, what=f"{w.name} tree {t} level {l}")
+    return otrees
+
+
+def check_walks(w, inp, tree, otrees, mode, p, k, n_keys, with_attention=True):
+    Z = zha()
+    sel, cnt, st = tree.search(inp.Q, MODE[mode], p, k, with_stats=True)
+    out, lse = tree.attend(inp.Q, sel, cnt, out_dtype=torch.float32)
+    tree.sync_status()
+    sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+    stats = Z.parse_stats(st)
+    out = host64(out).reshape(w.walks, w.d)
+    lse = lse.cpu().numpy()
+    checked = parted = 0
+    for (b, h), ot in otrees.items():
+        K = host64(inp.K[b, h, :n_keys])
+        V = host64(inp.V[b, h, :n_keys])
+        for wi, hq, i in walks_of_tree(w, b, h):
+            q = host64(inp.Q[b, hq, i])
+            ow = O.search(ot, q, MODE[mode], p, k, w.top_width)
+            if compare_selection(sel, cnt, {wi: ow}):
+                parted += 1
+                continue
+            assert stats[wi]["work"] == ow.work and stats[wi]["keys_read"] == ow.keys_read
+            if with_attention:
+                o_out, o_lse = O.attend(K, V, q, ow.sel, w.chunk, ot.n_nodes[1], w.beta)
+                assert_attention_close(out[wi], lse[wi], o_out, o_lse, 3e-3, f"{w.name} walk {wi}")
+            checked += 1
+    print(f"{w.name} {mode}: {checked} sampled walks match, {parted} part at oracle near-ties")
+    assert checked > 0
+
+
+def test_kv256k_full_with_appends():
+    w = S.WORKLOADS["kv256k"]
+    inp = S.draw(w, device="cuda")
+    Z = zha()
+    # the cache holds the appended keys already (drawn with it); appending writes them again
+    tree = Z.Tree(inp.K, inp.V, inp.refs, w.n_keys, w.chunk, w.depth, w.beta, w.top_width)
+    sample = [(0, 0), (w.batch - 1, w.n_kv_heads - 1)]
+    otrees = check_trees(w, inp, tree, sample)
+    check_walks(w, inp, tree, otrees, "top_p", 0.9, 0, w.n_keys)
+
+    new_k = inp.K[:, :, w.n_keys:].permute(2, 0, 1, 3).contiguous()
+    new_v = inp.V[:, :, w.n_keys:].permute(2, 0, 1, 3).contiguous()
+    for i in range(w.appends):
+        tree.append(new_k[i], new_v[i])
+    tree.sync_status()
+    assert tree.n_keys == w.capacity
+    assert tree.level_sizes() == w.level_sizes(w.capacity)
+    for key, ot in otrees.items():
+        O.append(ot, host64(inp.K[key[0], key[1]]), w.appends, threads=THREADS)
+    check_trees(w, inp, tree, sample, otrees=otrees)
+    check_walks(w, inp, tree, otrees, "top_p", 0.9, 0, w.capacity)
+    tree.close()
+
+
+def test_kv1m_full():
+    w = S.WORKLOADS["kv1m"]
+    inp = S.draw(w, device="cuda")
+    Z = zha()
+    tree = Z.Tree(inp.K, inp.V, inp.refs, w.n_keys, w.chunk, w.depth, w.beta, w.top_width)
+    otrees = check_trees(w, inp, tree, [(0, 0), (w.batch - 1, w.n_kv_heads - 1)])
+    for mode, p, k in w.modes:
+        check_walks(w, inp, tree, otrees, mode, p, k, w.n_keys)
+    tree.close()
+
+
+def test_prefill_sampled():
+    w = S.WORKLOADS["prefill256k"]
+    inp = S.draw(w, device="cuda")
+    Z = zha()
+    tree = Z.Tree(inp.K, inp.V, inp.refs, w.n_keys, w.chunk, w.depth, w.beta, w.top_width)
+    sel, cnt, st = tree.search(inp.Q, Z.TOP_P, 0.9, with_stats=True)
+    out, lse = tree.attend(inp.Q, sel, cnt, out_dtype=torch.float32)
+    tree.sync_status()
+    sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+    stats = Z.parse_stats(st)
+    out = host64(out).reshape(w.walks, w.d)
+    lse = lse.cpu().numpy()
+    rng = np.random.default_rng(3)
+    group = w.n_q_heads // w.n_kv_heads
+    otrees = {}
+    checked = parted = 0
+    for _ in range(64):
+        hq = int(rng.integers(w.n_q_heads))
+        i = int(rng.integers(w.queries_per_head))
+        h = hq // group
+        if h not in otrees:
+            otrees[h] = (oracle_tree(inp, 0, h, threads=THREADS), host64(inp.K[0, h, : w.n_keys]),
+                         host64(inp.V[0, h, : w.n_keys]))
+        ot, K, V = otrees[h]
+        wi = hq * w.queries_per_head + i
+        q = host64(inp.Q[0, hq, i])
+        ow = O.search(ot, q, O.TOP_P, 0.9, 0, w.top_width)
+        if compare_selection(sel, cnt, {wi: ow}):
+            parted += 1
+            continue
+        assert stats[wi]["work"] == ow.work
+        o_out, o_lse = O.attend(K, V, q, ow.sel, w.chunk, ot.n_nodes[1], w.beta)
+        assert_attention_close(out[wi], lse[wi], o_out, o_lse, 3e-3, f"prefill walk {wi}")
+        checked += 1
+    print(f"prefill: {checked} sampled walks match, {parted} part at oracle near-ties")
+    assert checked > 0
+    tree.close()

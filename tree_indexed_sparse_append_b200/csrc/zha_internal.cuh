@@ -23,19 +23,19 @@ __device__ __forceinline__ void report(int *status, int code) {
 // Loads. Node data is streamed once per launch: keep it out of L1.
 __device__ __forceinline__ float4 ld_stream4(const float *p) {
     float4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+    asm("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                  : "l"(p));
     return v;
 }
 __device__ __forceinline__ float2 ld_stream2(const float *p) {
     float2 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
+    asm("ld.global.nc.L1::no_allocate.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
     return v;
 }
 __device__ __forceinline__ uint4 ld_stream_u4(const void *p) {
     uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
@@ -118,8 +118,8 @@ __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x
 // one complete sum: that of row (lane >> (5 - log2 RP)). Each halving step
 // swaps half of the remaining values with the partner lane, so RP rows cost
 // RP - 1 + (5 - log2 RP) shuffles instead of 5 * RP.
-template <int RP>
-__device__ __forceinline__ float transpose_reduce(float (&v)[RP], int lane) {
+template <int RP, typename F = float>
+__device__ __forceinline__ F transpose_reduce(F (&v)[RP], int lane) {
     constexpr int LG = ilog2(RP);
 #pragma unroll
     for (int step = 0; step < LG; ++step) {
@@ -128,12 +128,12 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[RP], int lane) {
         const bool upper = (lane & off) != 0;
 #pragma unroll
         for (int i = 0; i < half; ++i) {
-            float send = upper ? v[i] : v[i + half];
-            float keep = upper ? v[i + half] : v[i];
+            F send = upper ? v[i] : v[i + half];
+            F keep = upper ? v[i + half] : v[i];
             v[i] = keep + __shfl_xor_sync(FULL, send, off);
         }
     }
-    float x = v[0];
+    F x = v[0];
 #pragma unroll
     for (int off = 16 >> LG; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
     return x;
