@@ -198,7 +198,7 @@ def oracle_sample(w, inp, n_trees: int, threads: int):
 
 
 # ---------------------------------------------------------------------------
-def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes):
+def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes, with_dense: bool = False):
     import torch
 
     import synthetic as S
@@ -309,6 +309,40 @@ def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes
                           "kernel_ms_per_step": {kk: v["ms"] / max(1, args.profile_steps) for kk, v in kt.items()},
                           "kernel_sum_ms_per_step": step_ms, "levels_walked": levels}
 
+    # the full-scan indexer on the same trees (the comparison the 1M workload asks for)
+    dense = None
+    if with_dense:
+        dense = {}
+        max_sel_d = tree.n_keys
+        dsel = torch.empty(Wk, max_sel_d, dtype=torch.int32, device=dev)
+        dcnt = torch.empty(Wk, dtype=torch.int32, device=dev)
+        for mname, p, k in modes:
+            mode = Z.TOP_P if mname == "top_p" else Z.TOP_K
+            for _ in range(3):
+                tree.dense_scan(inp.Q, mode, p, k, max_sel=max_sel_d, out=(dsel, dcnt))
+            ts = []
+            for _ in range(10):
+                flush.zero_()
+                e0.record(st)
+                tree.dense_scan(inp.Q, mode, p, k, max_sel=max_sel_d, out=(dsel, dcnt))
+                e1.record(st)
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            tree.sync_status()
+            ms = sorted(ts)[len(ts) // 2]
+            tree.profile(True)
+            flush.zero_()
+            tree.dense_scan(inp.Q, mode, p, k, max_sel=max_sel_d, out=(dsel, dcnt))
+            dk = {kk: round(v[1], 4) for kk, v in tree.profile_read().items() if v[0]}
+            tree.profile(False)
+            kbytes = B * H * tree.n_keys * d * inp.K.element_size()
+            r = results[mname]
+            search_ms = sum(r["kernel_ms_per_step"][k2] for k2 in ("search_init", "score", "select", "union"))
+            dense[mname] = {"ms": ms, "key_read_gbs": kbytes / (ms / 1e3) / 1e9, "kernel_ms": dk,
+                            "keys_selected_mean": float(dcnt.float().mean().item()),
+                            "tree_search_ms": search_ms, "dense_over_tree_search": ms / search_ms}
+        del dsel, dcnt
+
     # end to end through the public API with host buffers
     mname, p, k = modes[0]
     mode = Z.TOP_P if mname == "top_p" else Z.TOP_K
@@ -360,7 +394,7 @@ def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes
     del inp, new_k, new_v, flush
     torch.cuda.empty_cache()
     return {"w": w, "results": results, "e2e": e2e, "build_ms": build_ms, "baseline": baseline,
-            "n_keys_after": n_after}
+            "n_keys_after": n_after, "dense": dense}
 
 
 def config_of(w, label):
@@ -396,7 +430,7 @@ def main():
     extra = None
     if not args.no_extra:
         w4 = S.WORKLOADS["kv1m"]
-        x = run_decode(w4, args, rank, world, dev, False, "kv1m", w4.modes)
+        x = run_decode(w4, args, rank, world, dev, False, "kv1m", w4.modes, with_dense=True)
         extra = {"workload": "kv1m decode: 8 seq x 8 KV heads x 1,048,576 keys, 32 q-heads, d=128, bf16, C=16, "
                              "depth 5, R=8",
                  "build_ms": x["build_ms"],
@@ -404,7 +438,7 @@ def main():
                                "attend_roofline": r["attend_roofline"],
                                "kernel_ms_per_step": r["kernel_ms_per_step"], "clocks": r["clocks"]}
                            for m, r in x["results"].items()},
-                 "e2e": x["e2e"]}
+                 "e2e": x["e2e"], "dense_scan": x["dense"]}
     r = head["results"]["top_p"]
     line = {
         "metric": METRIC, "value": r["qps"], "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -181,6 +181,26 @@ int zha_attend(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_heads, 
                float *lse, void *stream);
 
 /*
+ * zha_dense_scan: the full-scan indexer the tree walk is compared with ([P3]:
+ * sparse attention indexers such as DeepSeek Sparse Attention score every token).
+ * Every key of the walk's tree is scored, s_j = beta*<q, k_j>, and the selection
+ * rule of one tree level is applied to the keys: softmax over all n keys, then the
+ * shortest prefix of the keys ordered by mass (descending, ties by ascending key
+ * index) whose mass reaches p (ZHA_TOP_P; p >= 1 takes every key), or the k first
+ * in that order (ZHA_TOP_K).
+ * Q:         [B][H_q][n_q][d] of q_dtype; at most 32 walks per tree
+ *            ((H_q / H_kv) * n_q <= 32).
+ * sel:       [walks][max_sel] int32: selected key indices, ascending.
+ * sel_count: [walks] int32.
+ * Scratch of 8 * walks * n bytes (+ the queries in fp32) is taken from the tree.
+ * Errors as zha_search; a walk selecting more than max_sel keys keeps the first
+ * max_sel (ascending) and makes zha_sync_status return ZHA_ERR_CAPACITY.
+ */
+int zha_dense_scan(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q,
+                   zha_mode mode, float p, int k, int *sel, int *sel_count, int max_sel,
+                   void *stream);
+
+/*
  * zha_reserve: allocate the search and attend scratch for up to max_walks walks
  * and selections of up to max_sel chunks now, so that later calls with at most
  * these sizes allocate nothing (e.g. before capturing them in a CUDA graph).

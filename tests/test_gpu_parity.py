@@ -343,3 +343,34 @@ def test_append_past_capacity_is_refused():
         tree.append(K[:, :, 0].contiguous(), V[:, :, 0].contiguous())
     assert e.value.code == Z.ERR_CAPACITY
     tree.close()
+
+
+# ---------------------------------------------------------------------------
+# the full-scan indexer
+
+
+class _Sel:
+    def __init__(self, sel, gap, sd):
+        self.sel, self.tie_gap, self.tie_sum = sel, gap, sd
+
+
+@pytest.mark.parametrize("N,d,dtype,Hq,nq", [(4096, 64, torch.float32, 1, 8), (3001, 128, torch.bfloat16, 4, 2),
+                                             (200000, 64, torch.float32, 2, 2), (65536, 128, torch.bfloat16, 4, 8)])
+def test_dense_scan_matches_oracle(N, d, dtype, Hq, nq):
+    Z = zha()
+    K, V, refs, Q = _tiny(N, C=8, depth=3, d=d, R=4, B=2, H=1, Hq=Hq, nq=nq, dtype=dtype, seed=N % 97)
+    beta = 1 / np.sqrt(d)
+    tree = Z.Tree(K, V, refs, N, 8, 3, beta)
+    Qh = host64(Q)
+    for mode, p, k in ((O.TOP_P, 0.9, 0), (O.TOP_P, 0.5, 0), (O.TOP_P, 1.0, 0), (O.TOP_K, 0, 16), (O.TOP_K, 0, 1)):
+        sel, cnt = tree.dense_scan(Q, mode, p, k)
+        tree.sync_status()
+        sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+        for b in range(2):
+            Kd = host64(K[b, 0, :N])
+            for hq in range(Hq):
+                for i in range(nq):
+                    wi = (b * Hq + hq) * nq + i
+                    s, gap, sd = O.dense_scan(Kd, Qh[b, hq, i], beta, mode, p, k)
+                    compare_selection(sel, cnt, {wi: _Sel(s, gap, sd)})
+    tree.close()

@@ -27,7 +27,8 @@ TOP_P, TOP_K = 0, 1
 # Every symbol include/zha.h declares.
 SYMBOLS = ("zha_build", "zha_append", "zha_search", "zha_attend", "zha_reserve", "zha_level",
            "zha_num_keys", "zha_sync_status", "zha_destroy", "zha_last_error", "zha_version",
-           "zha_profile", "zha_profile_read", "zha_kernel_launches", "zha_last_search_info")
+           "zha_profile", "zha_profile_read", "zha_kernel_launches", "zha_last_search_info",
+           "zha_dense_scan")
 KERNEL_KINDS = ("build", "append", "search_init", "score", "select", "attend_plan", "attend_partial",
                 "attend_combine", "union")
 
@@ -78,6 +79,7 @@ def lib():
         L.zha_search.argtypes = [vp, vp, i, i, i, i, f, i, vp, vp, i, vp, vp]
         L.zha_attend.argtypes = [vp, vp, i, i, i, vp, vp, i, vp, i, vp, vp]
         L.zha_reserve.argtypes = [vp, ll, i]
+        L.zha_dense_scan.argtypes = [vp, vp, i, i, i, i, f, i, vp, vp, i, vp]
         L.zha_level.argtypes = [vp, i, ctypes.POINTER(vp), ctypes.POINTER(ll), ctypes.POINTER(ll),
                                 ctypes.POINTER(i)]
         L.zha_num_keys.argtypes = [vp]
@@ -223,6 +225,23 @@ class Tree:
                                 _dev(sel_count, "sel_count"), sel.shape[1], _dev(out, "out"), _dtype_code(out),
                                 _dev(lse, "lse"), _stream(stream)))
         return out, lse
+
+    def dense_scan(self, Q: torch.Tensor, mode: int = TOP_P, p: float = 0.9, k: int = 1,
+                   max_sel: int | None = None, out=None, stream=None):
+        """Full-scan indexer: every key scored, top-p / top-K over keys.
+        Returns (sel [walks][max_sel] int32 key indices ascending, sel_count [walks])."""
+        B, Hq, nq, d = Q.shape
+        W = B * Hq * nq
+        if max_sel is None:
+            max_sel = max(1, self.n_keys)
+        if out is None:
+            sel = torch.empty(W, max_sel, dtype=torch.int32, device=Q.device)
+            cnt = torch.empty(W, dtype=torch.int32, device=Q.device)
+        else:
+            sel, cnt = out
+        _check(lib().zha_dense_scan(self._h, _dev(Q, "Q"), _dtype_code(Q), Hq, nq, mode, float(p), int(k),
+                                    _dev(sel, "sel"), _dev(cnt, "sel_count"), max_sel, _stream(stream)))
+        return sel, cnt
 
     def reserve(self, max_walks: int, max_sel: int) -> None:
         _check(lib().zha_reserve(self._h, int(max_walks), int(max_sel)))

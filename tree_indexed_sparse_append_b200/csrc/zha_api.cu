@@ -356,6 +356,47 @@ int zha_attend(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads, int
     return ZHA_OK;
 }
 
+int zha_dense_scan(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q, zha_mode mode, float p,
+                   int k, int *sel, int *sel_count, int max_sel, void *stream) {
+    long long W;
+    int G;
+    int rc = check_queries(t, Q, q_dtype, n_q_heads, n_q, &W, &G);
+    if (rc) return rc;
+    if (G > 32) return fail(ZHA_ERR_INVALID, "the full-scan indexer takes at most 32 walks per tree (got %d)", G);
+    if (!sel || !sel_count) return fail(ZHA_ERR_INVALID, "sel and sel_count must not be NULL");
+    if (max_sel < 1) return fail(ZHA_ERR_INVALID, "max_sel must be >= 1");
+    if (mode == ZHA_TOP_P) {
+        if (!(p > 0.f) || std::isnan(p)) return fail(ZHA_ERR_INVALID, "top-p needs p > 0 (got %g)", (double)p);
+    } else if (mode == ZHA_TOP_K) {
+        if (k < 1) return fail(ZHA_ERR_INVALID, "top-K needs k >= 1 (got %d)", k);
+    } else {
+        return fail(ZHA_ERR_INVALID, "mode must be ZHA_TOP_P or ZHA_TOP_K");
+    }
+    const long long N = t->n > 0 ? t->n : 1;
+    const size_t need = align_up(sizeof(float) * W * t->cfg.d) + align_up(sizeof(float) * W * N) +
+                        align_up(sizeof(uint32_t) * W * N);
+    if (need > t->dws_bytes) {
+        if (t->dws) cudaFree(t->dws);
+        t->dws = nullptr;
+        t->dws_bytes = 0;
+        cudaError_t e = cudaMalloc(&t->dws, need);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return cuda_fail(e, "allocating full-scan scratch");
+        }
+        t->dws_bytes = need;
+    }
+    char *b = static_cast<char *>(t->dws);
+    float *qf = reinterpret_cast<float *>(b);
+    float *S = reinterpret_cast<float *>(b + align_up(sizeof(float) * W * t->cfg.d));
+    uint32_t *gkey = reinterpret_cast<uint32_t *>(b + align_up(sizeof(float) * W * t->cfg.d) +
+                                                  align_up(sizeof(float) * W * N));
+    ZHA_CUDA(zha::launch_dense_scan(t, Q, q_dtype, G, W, mode, p, k, sel, sel_count, max_sel, qf, S, gkey,
+                                    static_cast<cudaStream_t>(stream)),
+             "launching the full-scan indexer");
+    return ZHA_OK;
+}
+
 int zha_reserve(zha_tree *t, long long max_walks, int max_sel) {
     if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");
     if (max_walks < 1 || max_sel < 1) return fail(ZHA_ERR_INVALID, "max_walks and max_sel must be >= 1");
@@ -461,6 +502,7 @@ void zha_destroy(zha_tree *t) {
         if (t->nodes[l]) cudaFree(t->nodes[l]);
     if (t->d_status) cudaFree(t->d_status);
     if (t->ws) cudaFree(t->ws);
+    if (t->dws) cudaFree(t->dws);
     delete t;
 }
 

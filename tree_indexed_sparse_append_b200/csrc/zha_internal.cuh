@@ -181,6 +181,10 @@ struct zha_tree {
     long long ws_walks;
     int ws_max_sel;
 
+    // scratch of the full-scan indexer (grown on demand)
+    void *dws;
+    size_t dws_bytes;
+
     // diagnostics
     struct zha_profiler *prof;  // NULL unless zha_profile(tree, 1)
     long long last_W;
@@ -220,6 +224,13 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
 cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zha_dtype q_dtype,
                           int G, long long W, const int *sel, const int *sel_count, int max_sel,
                           void *out, zha_dtype out_dtype, float *lse, cudaStream_t st);
+
+// Top-p / top-K over all N candidates of each walk (scores S [W][N]), ids out.
+cudaError_t launch_select_all(const zha_tree *t, const float *S, uint32_t *gkey, long long N, long long W, int G,
+                              int mode, float p, int k, int *sel, int *sel_count, int max_sel, cudaStream_t st);
+cudaError_t launch_dense_scan(const zha_tree *t, const void *Q, zha_dtype q_dtype, int G, long long W, int mode,
+                              float p, int k, int *sel, int *sel_count, int max_sel, float *qf, float *S,
+                              uint32_t *gkey, cudaStream_t st);
 
 int num_sms();
 

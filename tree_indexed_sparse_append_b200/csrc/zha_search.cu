@@ -492,53 +492,76 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
         }
     }
 
-    // opened = key above kstar, or equal to it and among the first cstar (by id);
-    // each thread owns a contiguous run of positions so that ranks follow ids
-    const long long per = (F + NT - 1) / NT;
-    const long long beg = min(F, tid * per), end = min(F, beg + per);
+    // opened = key above kstar, or equal to it and among the first cstar (by id).
+    // Each warp owns a contiguous region of positions and reads it 32 at a time
+    // (coalesced); ballots give the ranks inside a group of 32, one block scan
+    // over the warps' counts the rest, so ranks follow ids.
+    constexpr int NW = NT / 32;
+    const int lane = tid & 31, wid = tid >> 5;
+    const long long region = ((F + NW - 1) / NW + 31) & ~31LL;
+    const long long rbeg = min(F, (long long)wid * region), rend = min(F, rbeg + region);
+    const unsigned below = (1u << lane) - 1u;
     // ranks among keys equal to kstar matter only when some of them stay closed
     const bool split_tie = !open_all && cstar < eq_count;
-    unsigned eq_local = 0;
-    if (split_tie)
-        for (long long i = beg; i < end; ++i) eq_local += key_at(i) == kstar;
-    unsigned eq_base = split_tie ? block_incl_scan<NT, unsigned>(eq_local, sh_u32, nullptr) - eq_local : 0u;
-    unsigned open_local = 0;
+    unsigned eq_base = 0;
+    if (split_tie) {
+        unsigned eq_w = 0;
+        for (long long i0 = rbeg; i0 < rend; i0 += 32) {
+            const long long i = i0 + lane;
+            eq_w += __popc(__ballot_sync(FULL, i < rend && key_at(i) == kstar));
+        }
+        const unsigned v = lane == 0 ? eq_w : 0u;
+        eq_base = block_incl_scan<NT, unsigned>(v, sh_u32, nullptr) - v;
+        eq_base = __shfl_sync(FULL, eq_base, 0);
+    }
+    // is position i opened? `eq` is the number of keys equal to kstar before this group
+    auto opened = [&](long long i, unsigned eq, unsigned &eq_in_group) -> bool {
+        const bool in = i < rend;
+        if (open_all) {
+            eq_in_group = 0;
+            return in;
+        }
+        const uint32_t key = in ? key_at(i) : 0u;
+        const bool is_eq = in && key == kstar;
+        const unsigned eqm = __ballot_sync(FULL, is_eq);
+        eq_in_group = __popc(eqm);
+        return in && (key > kstar || (is_eq && eq + __popc(eqm & below) < cstar));
+    };
+    unsigned open_w = 0;
     {
-        unsigned eq = eq_base;
-        for (long long i = beg; i < end; ++i) {
-            bool o = open_all;
-            if (!open_all) {
-                const uint32_t key = key_at(i);
-                o = key > kstar || (key == kstar && eq < cstar);
-                eq += key == kstar;
-            }
-            open_local += o;
+        unsigned eq = eq_base, eqg;
+        for (long long i0 = rbeg; i0 < rend; i0 += 32) {
+            const bool o = opened(i0 + lane, eq, eqg);
+            open_w += __popc(__ballot_sync(FULL, o));
+            eq += eqg;
         }
     }
     unsigned n_open;
-    unsigned open_base = block_incl_scan<NT, unsigned>(open_local, sh_u32, &n_open) - open_local;
+    const unsigned v_open = lane == 0 ? open_w : 0u;
+    unsigned open_base = block_incl_scan<NT, unsigned>(v_open, sh_u32, &n_open) - v_open;
+    open_base = __shfl_sync(FULL, open_base, 0);
 
     // write the opened ids (ascending, since frontier positions ascend in id)
     {
-        unsigned eq = eq_base, rank = open_base;
         unsigned *M_tree = a.M_next ? a.M_next + (long long)t * a.words_next * a.G : nullptr;
         unsigned *U_tree = a.U_next ? a.U_next + (long long)t * a.words_next : nullptr;
-        for (long long i = beg; i < end; ++i) {
-            bool o = open_all;
-            if (!open_all) {
-                const uint32_t key = key_at(i);
-                o = key > kstar || (key == kstar && eq < cstar);
-                eq += key == kstar;
+        unsigned eq = eq_base, eqg, rank = open_base;
+        for (long long i0 = rbeg; i0 < rend; i0 += 32) {
+            const long long i = i0 + lane;
+            const bool o = opened(i, eq, eqg);
+            const unsigned om = __ballot_sync(FULL, o);
+            if (o) {
+                const unsigned r = rank + __popc(om & below);
+                const long long id = frontier_id(a, par, npar, i);
+                if (a.level == 1) {
+                    if (r < (unsigned)a.max_sel) a.sel[walk * a.max_sel + r] = (int)id;
+                } else {
+                    a.par_out[walk * a.Lstride + r] = (int)id;
+                    set_bits(M_tree, U_tree, a.G, g, id * a.C, id * a.C + a.C);
+                }
             }
-            if (!o) continue;
-            const long long id = frontier_id(a, par, npar, i);
-            if (a.level == 1) {
-                if (rank < (unsigned)a.max_sel) a.sel[walk * a.max_sel + rank] = (int)id;
-            } else {
-                a.par_out[walk * a.Lstride + rank] = (int)id;
-                set_bits(M_tree, U_tree, a.G, g, id * a.C, id * a.C + a.C);
-            }
-            ++rank;
+            rank += __popc(om);
+            eq += eqg;
         }
         if (a.level > 1 && a.n_orph_next > 0) {
             const long long lo = a.n_level_next - a.n_orph_next, hi = a.n_level_next;
@@ -613,6 +636,49 @@ cudaError_t launch_score_d(const zha_tree *t, const ScoreArgs &a, cudaStream_t s
 }
 
 }  // namespace
+
+cudaError_t launch_select_all(const zha_tree *t, const float *S, uint32_t *gkey, long long N, long long W, int G,
+                              int mode, float p, int k, int *sel, int *sel_count, int max_sel, cudaStream_t st) {
+    // every one of the N candidates (keys) is in the frontier: the start-level path
+    SelectArgs se{};
+    se.level = 1;
+    se.C = 1;
+    se.c_shift = 0;
+    se.R = t->cfg.R;
+    se.G = G;
+    se.start = 1;
+    se.n_level = N;
+    se.n_orph = 0;
+    se.n_orph_next = 0;
+    se.n_level_next = 0;
+    se.S = S;
+    se.Sstride = N;
+    se.par_in = nullptr;
+    se.par_out = nullptr;
+    se.Lstride = 0;
+    se.n_par_in = nullptr;
+    se.n_par_out = nullptr;
+    se.M_next = nullptr;
+    se.U_next = nullptr;
+    se.words_next = 0;
+    se.mode = mode;
+    se.p = p;
+    se.k = k;
+    se.sel = sel;
+    se.max_sel = max_sel;
+    se.sel_count = sel_count;
+    se.stats = nullptr;
+    se.tail = 0;
+    se.status = t->d_status;
+    se.gkey = gkey;
+    Probe pr(t, ZHA_K_SELECT, st);
+    if (N > 8192) {
+        se.smem_keys = std::min<long long>(N, 16384);
+        return launch_select<512>(se, W, st);
+    }
+    se.smem_keys = N;
+    return launch_select<256>(se, W, st);
+}
 
 cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zha_dtype q_dtype, int G,
                           long long W, int mode, float p, int k, int *sel, int *sel_count, int max_sel,
