@@ -268,6 +268,38 @@ long long zha_num_keys(const zha_tree *tree);
    first device-side error recorded since the last call (ZHA_OK if none). */
 int zha_sync_status(zha_tree *tree, void *stream);
 
+/*
+ * zha_attend_noalloc: zha_attend for callers that cannot let the library
+ * allocate device memory (no counterpart in the paper: it only changes where
+ * the attention's working memory comes from).
+ *
+ * zha_attend grows the tree's scratch with cudaMalloc when a call needs more
+ * than it holds. Some callers cannot allow that once they run: a server that
+ * gives all device memory to its own pool at start-up, or a latency-critical
+ * loop that cannot take the synchronisation cudaMalloc / cudaFree may cause.
+ * This call computes exactly what zha_attend computes (same arguments, same
+ * kernels, same results) but takes its scratch from one static device array of
+ * 32 MiB that the library holds on every GPU it is loaded on until the process
+ * exits. It calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Size limit: the scratch needed is about walks * min(128, ceil(C * (max_sel + 1)
+ * / 128)) * (4 * d + 12) bytes; a call needing more than 32 MiB fails with
+ * ZHA_ERR_CAPACITY and a message giving both sizes, launching nothing.
+ * First call: on each device, the first call looks the array's device address up
+ * (cudaGetSymbolAddress, with the tree's device current); make that first call
+ * before any stream capture.
+ * Sharing: every call on a device uses the same array, and each call overwrites
+ * what the last one left there. Calls that can overlap on the GPU (different
+ * streams, different trees, or different host threads without ordering) race on
+ * it and give wrong results: order them on one stream, or use zha_attend.
+ * Profiling (zha_profile) does not time this call; zha_kernel_launches counts it.
+ * Errors: as zha_attend, plus ZHA_ERR_CAPACITY (scratch limit above) and
+ * ZHA_ERR_INVALID when the current device is not the tree's.
+ */
+int zha_attend_noalloc(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q,
+                       const int *sel, const int *sel_count, int max_sel, void *out,
+                       zha_dtype out_dtype, float *lse, void *stream);
+
 /* Frees the tree's node storage and scratch. NULL is a no-op. Pending work that
    uses the tree must have finished. */
 void zha_destroy(zha_tree *tree);

@@ -28,7 +28,7 @@ TOP_P, TOP_K = 0, 1
 SYMBOLS = ("zha_build", "zha_append", "zha_search", "zha_attend", "zha_reserve", "zha_level",
            "zha_num_keys", "zha_sync_status", "zha_destroy", "zha_last_error", "zha_version",
            "zha_profile", "zha_profile_read", "zha_kernel_launches", "zha_last_search_info",
-           "zha_dense_scan")
+           "zha_dense_scan", "zha_attend_noalloc")
 KERNEL_KINDS = ("build", "append", "search_init", "score", "select", "attend_plan", "attend_partial",
                 "attend_combine", "union")
 
@@ -78,6 +78,7 @@ def lib():
         L.zha_append.argtypes = [vp, vp, vp, vp]
         L.zha_search.argtypes = [vp, vp, i, i, i, i, f, i, vp, vp, i, vp, vp]
         L.zha_attend.argtypes = [vp, vp, i, i, i, vp, vp, i, vp, i, vp, vp]
+        L.zha_attend_noalloc.argtypes = [vp, vp, i, i, i, vp, vp, i, vp, i, vp, vp]
         L.zha_reserve.argtypes = [vp, ll, i]
         L.zha_dense_scan.argtypes = [vp, vp, i, i, i, i, f, i, vp, vp, i, vp]
         L.zha_level.argtypes = [vp, i, ctypes.POINTER(vp), ctypes.POINTER(ll), ctypes.POINTER(ll),
@@ -224,6 +225,18 @@ class Tree:
         _check(lib().zha_attend(self._h, _dev(Q, "Q"), _dtype_code(Q), Hq, nq, _dev(sel, "sel"),
                                 _dev(sel_count, "sel_count"), sel.shape[1], _dev(out, "out"), _dtype_code(out),
                                 _dev(lse, "lse"), _stream(stream)))
+        return out, lse
+
+    def attend_noalloc(self, Q: torch.Tensor, sel: torch.Tensor, sel_count: torch.Tensor, out: torch.Tensor,
+                       lse: torch.Tensor | None = None, stream=None):
+        """attend() for callers whose device memory may not be allocated by the library:
+        zha_attend_noalloc uses a fixed static device array as scratch. The caller
+        provides out (and lse) already allocated; nothing is allocated here."""
+        B, Hq, nq, d = Q.shape
+        _check(lib().zha_attend_noalloc(self._h, _dev(Q, "Q"), _dtype_code(Q), Hq, nq, _dev(sel, "sel"),
+                                        _dev(sel_count, "sel_count"), sel.shape[1], _dev(out, "out"),
+                                        _dtype_code(out), _dev(lse, "lse") if lse is not None else None,
+                                        _stream(stream)))
         return out, lse
 
     def dense_scan(self, Q: torch.Tensor, mode: int = TOP_P, p: float = 0.9, k: int = 1,

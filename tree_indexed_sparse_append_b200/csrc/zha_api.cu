@@ -214,6 +214,12 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     return ZHA_OK;
 }
 
+// Records `msg` as the message zha_last_error returns on this host thread.
+int set_error(int code, const char *msg) {
+    g_error = msg;
+    return code;
+}
+
 }  // namespace zha
 
 extern "C" {

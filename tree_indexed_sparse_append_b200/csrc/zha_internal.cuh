@@ -212,6 +212,8 @@ struct Scratch {
 };
 
 int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s);
+// Records an error message for zha_last_error (this host thread); returns code.
+int set_error(int code, const char *msg);
 
 // kernel launchers (return cudaError_t of the launch)
 cudaError_t launch_build_level(const zha_tree *t, int level, long long j0, long long j1,
