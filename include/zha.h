@@ -282,8 +282,10 @@ int zha_sync_status(zha_tree *tree, void *stream);
  * 32 MiB that the library holds on every GPU it is loaded on until the process
  * exits. It calls no cudaMalloc, cudaFree or other allocating routine.
  *
- * Size limit: the scratch needed is about walks * min(128, ceil(C * (max_sel + 1)
- * / 128)) * (4 * d + 12) bytes; a call needing more than 32 MiB fails with
+ * Size limit: the scratch needed is (16,384 + walks) * 1.0625 * (4 * d + 20)
+ * + walks * (4 * d + 32) bytes, give or take alignment (9.5 MB at 256 walks and
+ * d = 128; 32 MiB holds about 21,000 walks at d = 128, 40,000 at d = 64 and
+ * 8,000 at d = 256); a call needing more than 32 MiB fails with
  * ZHA_ERR_CAPACITY and a message giving both sizes, launching nothing.
  * First call: on each device, the first call looks the array's device address up
  * (cudaGetSymbolAddress, with the tree's device current); make that first call

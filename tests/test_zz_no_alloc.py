@@ -95,12 +95,11 @@ def test_noalloc_refuses_more_than_its_scratch():
     w = W_SMALL
     inp = S.draw(w, device="cuda")
     tree = Z.Tree(inp.K, inp.V, inp.refs, w.n_keys, w.chunk, w.depth, w.beta, w.top_width)
-    # 512 walks of up to 513 chunks each: 128 items of 520 bytes per walk, 34 MB in all
-    n_q = 8
+    # 32,768 walks (512 queries per head) need 43.5 MB of scratch at d = 128
+    n_q = 512
     Q = queries(w, inp, n_q)
     walks = w.batch * w.n_q_heads * n_q
-    max_sel = tree.level(1)[1]
-    sel = torch.zeros(walks, max_sel, dtype=torch.int32, device="cuda")
+    sel = torch.zeros(walks, 1, dtype=torch.int32, device="cuda")
     cnt = torch.zeros(walks, dtype=torch.int32, device="cuda")
     out = torch.zeros(w.batch, w.n_q_heads, n_q, w.d, dtype=torch.float32, device="cuda")
     lse = torch.zeros(walks, dtype=torch.float32, device="cuda")

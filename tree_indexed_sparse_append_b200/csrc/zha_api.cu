@@ -138,18 +138,9 @@ void probe_end(const zha_tree *t, int kind, cudaStream_t st) {
 int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     const zha_config &c = t->cfg;
     const long long W = walks < 1 ? 1 : walks;
-    const int G = 0;  // layout below depends only on W and T
-    (void)G;
+    (void)max_sel;  // the layout depends on the walks and the tree only
     const long long cap1 = t->cap_nodes[1] > 0 ? t->cap_nodes[1] : 1;
     const long long cap2 = c.depth >= 2 && t->cap_nodes[2] > 0 ? t->cap_nodes[2] : 1;
-    // attend items: a walk's keys (at most C * (max_sel + 1)) in items of >= 128 keys,
-    // at most 128 items per walk (constants of zha_attend.cu)
-    const long long keys_max = (long long)c.chunk * ((long long)max_sel + 1);
-    long long per_walk_items = (keys_max + 127) / 128;
-    if (per_walk_items > 128) per_walk_items = 128;
-    if (per_walk_items < 1) per_walk_items = 1;
-    const long long max_items = W * per_walk_items;
-
     size_t off = 0;
     auto take = [&](size_t bytes) {
         size_t o = off;
@@ -171,10 +162,8 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     const size_t U_start = off;
     for (int l = 1; l <= c.depth; ++l) o_U[l] = take(sizeof(unsigned) * t->T * ((t->cap_nodes[l] + 31) / 32));
     const size_t U_bytes = off - U_start;
-    const size_t o_io = take(sizeof(int) * (W + 1));
-    const size_t o_iw = take(sizeof(int) * max_items);
-    const size_t o_wd = take(sizeof(int) * W);
-    const size_t o_pa = take(sizeof(float) * max_items * (c.d + 2));
+    const AttendLayout att = attend_layout(W, c.d);
+    const size_t o_att = take(att.bytes);
     const size_t need = off;
 
     if (need > t->ws_bytes) {
@@ -204,13 +193,9 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     s->U_base = reinterpret_cast<unsigned *>(b + U_start);
     s->M_bytes = M_bytes;
     s->U_bytes = U_bytes;
-    s->item_off = reinterpret_cast<int *>(b + o_io);
-    s->item_walk = reinterpret_cast<int *>(b + o_iw);
-    s->walk_done = reinterpret_cast<int *>(b + o_wd);
-    s->partial = reinterpret_cast<float *>(b + o_pa);
+    attend_carve(att, b + o_att, s);
     s->Sstride = cap1;
     s->Lstride = cap2;
-    s->max_items = max_items;
     return ZHA_OK;
 }
 

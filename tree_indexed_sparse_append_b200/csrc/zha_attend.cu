@@ -9,19 +9,24 @@
 //   out = sum_i softmax_i(beta <q, k_i>) v_i,   lse = logsumexp_i(beta <q, k_i>).
 //
 // Design (split-K decode attention, fp32 accumulation, two launches):
-//   attend_plan   one CTA scans the walks' key counts into item offsets and an
-//                 item -> walk map; a walk's key list is cut into at most
-//                 MAX_SPLIT items of at least SEG keys. Walks without keys get
-//                 out = 0, lse = -inf here.
+//   attend_plan   one CTA sums the walks' key counts, sets the item length from
+//                 that total so that the whole call has at most ITEM_BUDGET
+//                 items (never fewer than SEG_MIN keys each, never more than
+//                 MAX_SPLIT items per walk), and scans the walks' item and group
+//                 counts into offsets and an item -> walk map. Walks without
+//                 keys get out = 0, lse = -inf here.
 //   attend_items  grid-stride over items, one warp per item. The item's chunk
-//                 ids are loaded once (one per lane) and broadcast by shuffle.
-//                 A row of K or V is read with 16-byte loads by LPR lanes (16 for
-//                 d = 128 bf16), so a warp step covers KPW = 32/LPR keys; U steps
-//                 of K and V rows are issued before any is used, their U dot
-//                 products are independent, and the online softmax takes them in
-//                 one update. The warp that finishes a walk's last item (an
-//                 atomic ticket after a fence; nobody waits) merges the walk's
-//                 partial results by log-sum-exp and writes out and lse.
+//                 ids come through a two-window register prefetch (32 ids per
+//                 window, one per lane) and are broadcast by shuffle. A row of K
+//                 or V is read with 16-byte loads by LPR lanes (16 for d = 128
+//                 bf16), so a warp step covers KPW = 32/LPR keys; U steps of K
+//                 and V rows are issued before any is used, their U dot products
+//                 are independent, and the online softmax takes them in one
+//                 update. A walk's items form groups of GROUP: the warp that
+//                 finishes a group's last item (an atomic ticket after a fence;
+//                 nobody waits) merges the group by log-sum-exp, and the warp
+//                 that finishes a walk's last group merges the groups and writes
+//                 out and lse. Merges read their rows in one or two round trips.
 // fp32 caches take their dot products in fp64.
 #include <cmath>
 #include <type_traits>
@@ -31,8 +36,10 @@
 namespace zha {
 namespace {
 
-constexpr int SEG = 128;        // keys per work item, at least
-constexpr int MAX_SPLIT = 128;  // work items per walk, at most
+constexpr int SEG_MIN = 128;         // keys per work item, at least
+constexpr int MAX_SPLIT = 512;       // work items per walk, at most
+constexpr int ITEM_BUDGET = 16384;   // work items per call (before per-walk rounding)
+constexpr int GROUP = 16;            // items merged together first
 
 __device__ __forceinline__ long long walk_keys(const int *sel_count, long long w, int max_sel, int C,
                                                long long tail) {
@@ -41,9 +48,10 @@ __device__ __forceinline__ long long walk_keys(const int *sel_count, long long w
     return (long long)C * c + tail;
 }
 
-__device__ __forceinline__ long long seg_len(long long L) {
-    long long s = (L + MAX_SPLIT - 1) / MAX_SPLIT;
-    return s > SEG ? s : SEG;
+// Keys per item of a walk of L keys, given the call's item length.
+__device__ __forceinline__ long long seg_len(long long L, long long seg) {
+    const long long s = (L + MAX_SPLIT - 1) / MAX_SPLIT;
+    return s > seg ? s : seg;
 }
 
 template <typename OT>
@@ -55,47 +63,92 @@ struct PlanArgs {
     const int *sel_count;
     int max_sel, C, D, out_bf16;
     long long tail, W;
-    int *item_off;
-    int *item_walk;
-    int *walk_done;
+    int *item_off;    // [W + 1]
+    int *group_off;   // [W + 1]
+    int *seg;         // [1] keys per item of the call (before the per-walk cap)
+    int *item_walk;   // [items]
+    int *walk_done;   // [W]
+    int *group_done;  // [groups]
     void *out;
     float *lse;
 };
 
-__global__ void __launch_bounds__(1024) attend_plan_kernel(PlanArgs a) {
-    __shared__ long long sh[32];
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    long long carry = 0;
-    for (long long base = 0; base < a.W; base += blockDim.x) {
-        const long long w = base + threadIdx.x;
-        long long items = 0;
-        if (w < a.W) {
-            const long long L = walk_keys(a.sel_count, w, a.max_sel, a.C, a.tail);
-            items = L > 0 ? (L + seg_len(L) - 1) / seg_len(L) : 0;
+// Block-wide inclusive scan of two counts (1024 threads); returns the totals.
+__device__ __forceinline__ void block_scan2(long long &a, long long &b, long long *sh, long long &ta,
+                                            long long &tb) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long ya = __shfl_up_sync(FULL, a, o), yb = __shfl_up_sync(FULL, b, o);
+        if (lane >= o) {
+            a += ya;
+            b += yb;
         }
-        long long inc = items;
+    }
+    if (lane == 31) {
+        sh[wid] = a;
+        sh[32 + wid] = b;
+    }
+    __syncthreads();
+    if (wid == 0) {
+        long long x = lane < nw ? sh[lane] : 0, y = lane < nw ? sh[32 + lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            long long y = __shfl_up_sync(FULL, inc, o);
-            if (lane >= o) inc += y;
-        }
-        if (lane == 31) sh[wid] = inc;
-        __syncthreads();
-        if (wid == 0) {
-            long long s = lane < (int)(blockDim.x >> 5) ? sh[lane] : 0;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                long long y = __shfl_up_sync(FULL, s, o);
-                if (lane >= o) s += y;
+            const long long yx = __shfl_up_sync(FULL, x, o), yy = __shfl_up_sync(FULL, y, o);
+            if (lane >= o) {
+                x += yx;
+                y += yy;
             }
-            sh[lane] = s;
         }
-        __syncthreads();
-        const long long excl = carry + (wid > 0 ? sh[wid - 1] : 0) + inc - items;
+        sh[lane] = x;
+        sh[32 + lane] = y;
+    }
+    __syncthreads();
+    if (wid > 0) {
+        a += sh[wid - 1];
+        b += sh[32 + wid - 1];
+    }
+    ta = sh[nw - 1];
+    tb = sh[32 + nw - 1];
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(1024) attend_plan_kernel(PlanArgs a) {
+    __shared__ long long sh[64];
+    // 1. the call's total key count sets the item length
+    long long keys = 0;
+    for (long long w = threadIdx.x; w < a.W; w += blockDim.x)
+        keys += walk_keys(a.sel_count, w, a.max_sel, a.C, a.tail);
+    {
+        long long zero = 0, total = 0, unused = 0;
+        block_scan2(keys, zero, sh, total, unused);
+        keys = total;
+    }
+    long long seg = (keys + ITEM_BUDGET - 1) / ITEM_BUDGET;
+    if (seg < SEG_MIN) seg = SEG_MIN;
+    if (seg > (1LL << 30)) seg = 1LL << 30;
+    if (threadIdx.x == 0) a.seg[0] = (int)seg;
+
+    // 2. items and groups per walk, scanned into offsets
+    long long icarry = 0, gcarry = 0;
+    for (long long base = 0; base < a.W; base += blockDim.x) {
+        const long long w = base + threadIdx.x;
+        long long items = 0, groups = 0;
         if (w < a.W) {
-            a.item_off[w] = (int)excl;
+            const long long L = walk_keys(a.sel_count, w, a.max_sel, a.C, a.tail);
+            const long long sw = seg_len(L, seg);
+            items = L > 0 ? (L + sw - 1) / sw : 0;
+            groups = (items + GROUP - 1) / GROUP;
+        }
+        long long iinc = items, ginc = groups, itot, gtot;
+        block_scan2(iinc, ginc, sh, itot, gtot);
+        if (w < a.W) {
+            const long long i0 = icarry + iinc - items, g0 = gcarry + ginc - groups;
+            a.item_off[w] = (int)i0;
+            a.group_off[w] = (int)g0;
             a.walk_done[w] = 0;
-            for (long long i = 0; i < items; ++i) a.item_walk[excl + i] = (int)w;
+            for (long long i = 0; i < items; ++i) a.item_walk[i0 + i] = (int)w;
+            for (long long g = 0; g < groups; ++g) a.group_done[g0 + g] = 0;
             if (items == 0) {  // no key at all: out = 0, lse = -inf
                 for (int e = 0; e < a.D; ++e) {
                     if (a.out_bf16) store_out(static_cast<__nv_bfloat16 *>(a.out) + w * a.D + e, 0.f);
@@ -104,22 +157,26 @@ __global__ void __launch_bounds__(1024) attend_plan_kernel(PlanArgs a) {
                 if (a.lse) a.lse[w] = -INFINITY;
             }
         }
-        carry += sh[(blockDim.x >> 5) - 1];
-        __syncthreads();
+        icarry += itot;
+        gcarry += gtot;
     }
-    if (threadIdx.x == 0) a.item_off[a.W] = (int)carry;
+    if (threadIdx.x == 0) {
+        a.item_off[a.W] = (int)icarry;
+        a.group_off[a.W] = (int)gcarry;
+    }
 }
 
 struct ItemArgs {
     const void *K, *V, *Q;
     int q_bf16, out_bf16;
-    const int *sel, *sel_count, *item_off, *item_walk;
-    int *walk_done;
+    const int *sel, *sel_count, *item_off, *group_off, *seg, *item_walk;
+    int *walk_done, *group_done;
     int max_sel, C, G;
     int c_shift;  // log2(C) when C is a power of two, else -1
     long long W, cap, n1, tail;
     float beta;
-    float *partial;  // [items][D + 2]: acc[D], m, l
+    float *partial;   // [items][D + 4]: acc[D], m, l (rows 16-byte aligned)
+    float *gpartial;  // [groups][D + 4]: the same, per group
     void *out;
     float *lse;
     int *status;
@@ -154,34 +211,68 @@ struct Row<float> {
     }
 };
 
-// Merges the partial results of one walk (one warp) and writes out / lse.
-template <int D>
-__device__ void combine_walk(const ItemArgs &a, long long walk, int lane) {
-    constexpr int CPL = D / 32;
-    const long long i0 = a.item_off[walk], i1 = a.item_off[walk + 1];
-    float m = -INFINITY;
-    for (long long i = i0 + lane; i < i1; i += 32) m = fmaxf(m, __ldcg(a.partial + i * (D + 2) + D));
-    m = warp_max(m);
-    float l = 0.f;
-    for (long long i = i0 + lane; i < i1; i += 32) {
-        const float mi = __ldcg(a.partial + i * (D + 2) + D);
-        if (mi != -INFINITY) l += __ldcg(a.partial + i * (D + 2) + D + 1) * expf(mi - m);
+// Loads the CPL consecutive floats of a partial row that one lane holds.
+template <int CPL>
+__device__ __forceinline__ void ld_cols(const float *p, float (&x)[CPL]) {
+    if constexpr (CPL == 2) {
+        const float2 v = __ldcg(reinterpret_cast<const float2 *>(p));
+        x[0] = v.x;
+        x[1] = v.y;
+    } else {
+#pragma unroll
+        for (int c = 0; c < CPL; c += 4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(p + c));
+            x[c] = v.x;
+            x[c + 1] = v.y;
+            x[c + 2] = v.z;
+            x[c + 3] = v.w;
+        }
     }
-    l = warp_sum(l);
-    float o[CPL];
+}
+
+// Merges n <= 32 partial rows (acc[D], m, l; stride D + 4) by log-sum-exp, in row
+// order. Lane i reads row i's (m, l); every row's acc is read before any is used
+// (RB rows at a time). The merged acc columns lane*CPL .. lane*CPL + CPL - 1 come
+// back in o.
+template <int D>
+__device__ __forceinline__ void merge_rows(const float *rows, int n, int lane, float &m, float &l,
+                                           float (&o)[D / 32]) {
+    constexpr int CPL = D / 32, PS = D + 4, RB = D >= 256 ? 8 : 16;
+    float mi = -INFINITY, li = 0.f;
+    if (lane < n) {
+        mi = __ldcg(rows + lane * PS + D);
+        li = __ldcg(rows + lane * PS + D + 1);
+    }
+    m = warp_max(mi);
+    const float wi = mi == -INFINITY ? 0.f : expf(mi - m);
+    l = warp_sum(wi * li);
 #pragma unroll
     for (int c = 0; c < CPL; ++c) o[c] = 0.f;
-#pragma unroll 4
-    for (long long i = i0; i < i1; ++i) {
-        const float *pi = a.partial + i * (D + 2);
-        const float mi = __ldcg(pi + D);
-        float x[CPL];
+    for (int i0 = 0; i0 < n; i0 += RB) {
+        float x[RB][CPL];
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) x[c] = __ldcg(pi + lane * CPL + c);
-        const float w = mi == -INFINITY ? 0.f : expf(mi - m);
+        for (int j = 0; j < RB; ++j) {
+            if (i0 + j < n) {
+                ld_cols<CPL>(rows + (i0 + j) * PS + lane * CPL, x[j]);
+            } else {
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) o[c] = fmaf(w, x[c], o[c]);
+                for (int c = 0; c < CPL; ++c) x[j][c] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+            const float w = __shfl_sync(FULL, wi, (i0 + j) & 31);
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) o[c] = fmaf(w, x[j][c], o[c]);
+        }
     }
+}
+
+// Writes a walk's normalised output (lane's columns lane*CPL ..) and lse.
+template <int D>
+__device__ __forceinline__ void write_out(const ItemArgs &a, long long walk, int lane, float m, float l,
+                                          const float (&o)[D / 32]) {
+    constexpr int CPL = D / 32;
     const bool empty = !(l > 0.f);
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
@@ -201,6 +292,8 @@ __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
     constexpr int KPW = 32 / LPR;                // keys per warp step
     constexpr int COLS = EPL * VPL;
     constexpr int U = VPL == 1 ? 8 : 4;          // steps whose rows are in flight together
+    constexpr int CPL = D / 32, PS = D + 4;
+    static_assert(KPW * U <= 32, "one step must span fewer than 32 chunks of C >= 2 keys");
     using Dot = typename std::conditional<sizeof(T) == 4, double, float>::type;
     using Raw = typename Row<T>::Raw;
 
@@ -209,6 +302,7 @@ __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
     const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
     const long long total = a.item_off[a.W];
+    const long long seg = a.seg[0];
     const T *Kb = static_cast<const T *>(a.K);
     const T *Vb = static_cast<const T *>(a.V);
 
@@ -216,19 +310,22 @@ __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
         const long long walk = a.item_walk[item];
         const long long tree = walk / a.G;
         const long long L = walk_keys(a.sel_count, walk, a.max_sel, a.C, a.tail);
-        const long long seg = seg_len(L);
-        const long long k0 = (item - a.item_off[walk]) * seg;
-        const long long k1 = k0 + seg < L ? k0 + seg : L;
+        const long long i_first = a.item_off[walk];
+        const int nitems = a.item_off[walk + 1] - (int)i_first;
+        const long long sw = seg_len(L, seg);
+        const long long k0 = (item - i_first) * sw;
+        const long long k1 = k0 + sw < L ? k0 + sw : L;
         const long long nsel = L - a.tail;  // keys coming from selected chunks
         const int *wsel = a.sel + walk * a.max_sel;
 
-        // the segment's chunk ids, one per lane, when they fit in a warp
+        // chunk ids of the item, 32 per window, one per lane; the next window is
+        // loaded while the current one is used
         const long long ke = k1 < nsel ? k1 : nsel;
-        const long long c0 = k0 / a.C;
-        const long long c1 = ke > k0 ? (ke - 1) / a.C + 1 : c0;
-        const bool pre = c1 - c0 <= 32;
-        int my_chunk = 0;
-        if (pre && c0 + lane < c1) my_chunk = __ldg(wsel + c0 + lane);
+        const int c0 = (int)(k0 / a.C);
+        const int c1 = ke > k0 ? (int)((ke - 1) / a.C) + 1 : c0;
+        int wb = c0;
+        int cur = wb + lane < c1 ? __ldg(wsel + wb + lane) : 0;
+        int nxt = wb + 32 + lane < c1 ? __ldg(wsel + wb + 32 + lane) : 0;
 
         float q[COLS];
 #pragma unroll
@@ -247,9 +344,16 @@ __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
         // key positions fit in 32 bits (at most C * (max_sel + 1) per walk)
         const T *Kt = Kb + tree * a.cap * D;
         const T *Vt = Vb + tree * a.cap * D;
-        const int nsel32 = (int)nsel, k1_32 = (int)k1, c0_32 = (int)c0, C = a.C;
+        const int nsel32 = (int)nsel, k1_32 = (int)k1, C = a.C;
         const int tail0 = (int)(a.n1 * a.C);
         for (int kb = (int)k0; kb < k1_32; kb += KPW * U) {
+            // a step spans fewer than 32 chunks, so one shift keeps it inside cur + nxt
+            const int cfirst = a.c_shift >= 0 ? kb >> a.c_shift : kb / C;
+            if (cfirst - wb >= 32) {
+                wb += 32;
+                cur = nxt;
+                nxt = wb + 32 + lane < c1 ? __ldg(wsel + wb + 32 + lane) : 0;
+            }
             bool valid[U];
             int kid[U];
 #pragma unroll
@@ -259,12 +363,10 @@ __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
                 kid[u] = 0;
                 const int ci = a.c_shift >= 0 ? kk >> a.c_shift : kk / C;
                 const int co = a.c_shift >= 0 ? kk & (C - 1) : kk - ci * C;
-                int c = 0;
-                if (pre) {
-                    c = __shfl_sync(FULL, my_chunk, (ci - c0_32) & 31);
-                } else if (valid[u] && kk < nsel32) {
-                    c = __ldg(wsel + ci);
-                }
+                const int rel = ci - wb;
+                const int from_cur = __shfl_sync(FULL, cur, rel & 31);
+                const int from_nxt = __shfl_sync(FULL, nxt, rel & 31);
+                const int c = rel < 32 ? from_cur : from_nxt;
                 if (valid[u]) {
                     if (kk < nsel32) {
                         if (c < 0 || c >= a.n1) {
@@ -337,8 +439,26 @@ __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
             l = l * s1 + l2 * s2;
             m = mn;
         }
+
+        if (nitems == 1) {  // the walk is this item: write the result directly
+            if (grp == 0) {
+                const bool empty = !(l > 0.f);
+#pragma unroll
+                for (int v = 0; v < VPL; ++v)
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) {
+                        const long long col = walk * D + (v * LPR + gl) * EPL + e;
+                        const float r = empty ? 0.f : acc[v * EPL + e] / l;
+                        if (a.out_bf16) store_out(static_cast<__nv_bfloat16 *>(a.out) + col, r);
+                        else store_out(static_cast<float *>(a.out) + col, r);
+                    }
+                if (gl == 0 && a.lse) a.lse[walk] = empty ? -INFINITY : m + logf(l);
+            }
+            continue;
+        }
+
         if (grp == 0) {
-            float *out = a.partial + item * (D + 2);
+            float *out = a.partial + item * PS;
 #pragma unroll
             for (int v = 0; v < VPL; ++v)
 #pragma unroll
@@ -348,16 +468,40 @@ __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
                 out[D + 1] = l;
             }
         }
-        // the warp that completes a walk's last item merges the walk
+        // the warp that completes a group merges it; the one that completes the
+        // walk's last group merges the groups
         __threadfence();
         __syncwarp();
+        const int j = (int)(item - i_first), g = j / GROUP;
+        const int gsize = nitems - g * GROUP < GROUP ? nitems - g * GROUP : GROUP;
+        const long long g_first = a.group_off[walk];
+        const int ngroups = a.group_off[walk + 1] - (int)g_first;
         int ticket = 0;
+        if (lane == 0) ticket = atomicAdd(a.group_done + g_first + g, 1) + 1;
+        ticket = __shfl_sync(FULL, ticket, 0);
+        if (ticket != gsize) continue;
+        __threadfence();
+        float gm, gsum, o[CPL];
+        merge_rows<D>(a.partial + (i_first + (long long)g * GROUP) * PS, gsize, lane, gm, gsum, o);
+        if (ngroups == 1) {
+            write_out<D>(a, walk, lane, gm, gsum, o);
+            continue;
+        }
+        float *gp = a.gpartial + (g_first + g) * PS;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) gp[lane * CPL + c] = o[c];
+        if (lane == 0) {
+            gp[D] = gm;
+            gp[D + 1] = gsum;
+        }
+        __threadfence();
+        __syncwarp();
         if (lane == 0) ticket = atomicAdd(a.walk_done + walk, 1) + 1;
         ticket = __shfl_sync(FULL, ticket, 0);
-        if (ticket == a.item_off[walk + 1] - a.item_off[walk]) {
-            __threadfence();
-            combine_walk<D>(a, walk, lane);
-        }
+        if (ticket != ngroups) continue;
+        __threadfence();
+        merge_rows<D>(a.gpartial + g_first * PS, ngroups, lane, gm, gsum, o);
+        write_out<D>(a, walk, lane, gm, gsum, o);
     }
 }
 
@@ -380,6 +524,43 @@ cudaError_t launch_items(const zha_tree *t, const ItemArgs &ia, long long max_it
 
 }  // namespace
 
+AttendLayout attend_layout(long long W, int D) {
+    AttendLayout L{};
+    const long long w = W < 1 ? 1 : W;
+    L.max_items = ITEM_BUDGET + w;
+    L.max_groups = L.max_items / GROUP + w;
+    const long long ps = D + 4;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = (off + bytes + 255) & ~size_t(255);
+        return o;
+    };
+    L.item_off = take(sizeof(int) * (w + 1));
+    L.group_off = take(sizeof(int) * (w + 1));
+    L.seg = take(sizeof(int));
+    L.item_walk = take(sizeof(int) * L.max_items);
+    L.walk_done = take(sizeof(int) * w);
+    L.group_done = take(sizeof(int) * L.max_groups);
+    L.partial = take(sizeof(float) * L.max_items * ps);
+    L.gpartial = take(sizeof(float) * L.max_groups * ps);
+    L.bytes = off;
+    return L;
+}
+
+void attend_carve(const AttendLayout &L, void *base, Scratch *s) {
+    char *b = static_cast<char *>(base);
+    s->item_off = reinterpret_cast<int *>(b + L.item_off);
+    s->group_off = reinterpret_cast<int *>(b + L.group_off);
+    s->seg = reinterpret_cast<int *>(b + L.seg);
+    s->item_walk = reinterpret_cast<int *>(b + L.item_walk);
+    s->walk_done = reinterpret_cast<int *>(b + L.walk_done);
+    s->group_done = reinterpret_cast<int *>(b + L.group_done);
+    s->partial = reinterpret_cast<float *>(b + L.partial);
+    s->gpartial = reinterpret_cast<float *>(b + L.gpartial);
+    s->max_items = L.max_items;
+}
+
 cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zha_dtype q_dtype, int G,
                           long long W, const int *sel, const int *sel_count, int max_sel, void *out,
                           zha_dtype out_dtype, float *lse, cudaStream_t st) {
@@ -393,8 +574,11 @@ cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zh
     pl.tail = t->n - (long long)c.chunk * t->n_nodes[1];
     pl.W = W;
     pl.item_off = s.item_off;
+    pl.group_off = s.group_off;
+    pl.seg = s.seg;
     pl.item_walk = s.item_walk;
     pl.walk_done = s.walk_done;
+    pl.group_done = s.group_done;
     pl.out = out;
     pl.lse = lse;
     {
@@ -413,8 +597,11 @@ cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zh
     ia.sel = sel;
     ia.sel_count = sel_count;
     ia.item_off = s.item_off;
+    ia.group_off = s.group_off;
+    ia.seg = s.seg;
     ia.item_walk = s.item_walk;
     ia.walk_done = s.walk_done;
+    ia.group_done = s.group_done;
     ia.max_sel = max_sel;
     ia.C = c.chunk;
     ia.c_shift = (c.chunk & (c.chunk - 1)) == 0 ? __builtin_ctz((unsigned)c.chunk) : -1;
@@ -425,6 +612,7 @@ cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zh
     ia.tail = pl.tail;
     ia.beta = c.sharpness;
     ia.partial = s.partial;
+    ia.gpartial = s.gpartial;
     ia.out = out;
     ia.lse = lse;
     ia.status = t->d_status;

@@ -205,13 +205,27 @@ struct Scratch {
     size_t M_bytes, U_bytes;
     unsigned *M_base, *U_base;
     int *item_off;             // [W + 1] attend items per walk (prefix)
+    int *group_off;            // [W + 1] attend item groups per walk (prefix)
+    int *seg;                  // [1] keys per attend item of the call
     int *item_walk;            // [max_items] walk of each attend item
-    int *walk_done;            // [W] attend items finished per walk
-    float *partial;            // [max_items][D + 2]
+    int *walk_done;            // [W] attend groups finished per walk
+    int *group_done;           // [max_groups] attend items finished per group
+    float *partial;            // [max_items][D + 4]
+    float *gpartial;           // [max_groups][D + 4]
     long long Sstride, Lstride, max_items;
 };
 
 int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s);
+
+// Byte offsets of the attention's scratch for W walks of head dimension D, in
+// one block of `bytes` (offsets 256-byte aligned); its size depends on W and D only.
+struct AttendLayout {
+    size_t item_off, group_off, seg, item_walk, walk_done, group_done, partial, gpartial, bytes;
+    long long max_items, max_groups;
+};
+AttendLayout attend_layout(long long W, int D);
+// Points the attention fields of s into the block at base laid out by L.
+void attend_carve(const AttendLayout &L, void *base, Scratch *s);
 // Records an error message for zha_last_error (this host thread); returns code.
 int set_error(int code, const char *msg);
 

@@ -29,8 +29,6 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[ZHA_NOALLOC_SCR
 std::mutex g_addr_mu;
 void *g_addr[MAX_DEVICES];  // device address of g_noalloc_scratch, per device
 
-size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
-
 // Device address of the array on the current device; looked up on the first call.
 int scratch_address(int dev, void **out) {
     std::lock_guard<std::mutex> lock(g_addr_mu);
@@ -66,29 +64,14 @@ extern "C" int zha_attend_noalloc(zha_tree *t, const void *Q, zha_dtype q_dtype,
     const long long W = (long long)t->cfg.batch * n_q_heads * n_q;
     if (W > (1LL << 31) - 1 || G > (1LL << 30)) return zha::set_error(ZHA_ERR_INVALID, "too many walks");
 
-    // The attention's scratch, laid out as zha_attend lays it out: a walk's keys
-    // (at most C * (max_sel + 1)) are cut into items of at least 128 keys, at most
-    // 128 items per walk, and every item leaves d + 2 floats of partial result.
-    const long long keys_max = (long long)t->cfg.chunk * ((long long)max_sel + 1);
-    long long per_walk_items = (keys_max + 127) / 128;
-    if (per_walk_items > 128) per_walk_items = 128;
-    if (per_walk_items < 1) per_walk_items = 1;
-    const long long max_items = W * per_walk_items;
-    size_t need = 0;
-    const size_t o_item_off = need;
-    need = round256(need + sizeof(int) * (W + 1));
-    const size_t o_item_walk = need;
-    need = round256(need + sizeof(int) * max_items);
-    const size_t o_walk_done = need;
-    need = round256(need + sizeof(int) * W);
-    const size_t o_partial = need;
-    need = round256(need + sizeof(float) * max_items * (t->cfg.d + 2));
-    if (need > ZHA_NOALLOC_SCRATCH_BYTES) {
+    // the attention's scratch, laid out as zha_attend lays it out
+    const zha::AttendLayout layout = zha::attend_layout(W, t->cfg.d);
+    if (layout.bytes > ZHA_NOALLOC_SCRATCH_BYTES) {
         char msg[320];
         snprintf(msg, sizeof msg,
-                 "zha_attend_noalloc: %lld walks with max_sel %d need %zu bytes of scratch, more than the "
-                 "%zu of its static array; use zha_attend, fewer walks per call or a smaller max_sel",
-                 W, max_sel, need, ZHA_NOALLOC_SCRATCH_BYTES);
+                 "zha_attend_noalloc: %lld walks need %zu bytes of scratch, more than the %zu of its "
+                 "static array; use zha_attend or fewer walks per call",
+                 W, layout.bytes, ZHA_NOALLOC_SCRATCH_BYTES);
         return zha::set_error(ZHA_ERR_CAPACITY, msg);
     }
 
@@ -104,16 +87,11 @@ extern "C" int zha_attend_noalloc(zha_tree *t, const void *Q, zha_dtype q_dtype,
     int rc = scratch_address(dev, &base);
     if (rc) return rc;
 
-    char *b = static_cast<char *>(base);
     zha::Scratch s{};
-    s.item_off = reinterpret_cast<int *>(b + o_item_off);
-    s.item_walk = reinterpret_cast<int *>(b + o_item_walk);
-    s.walk_done = reinterpret_cast<int *>(b + o_walk_done);
-    s.partial = reinterpret_cast<float *>(b + o_partial);
-    s.max_items = max_items;
-    // The plan kernel writes every item offset and item owner the item kernel reads
-    // and zeroes the per-walk completion counters, so what an earlier call left in
-    // the array needs no clearing here.
+    zha::attend_carve(layout, base, &s);
+    // The plan kernel writes every offset, item owner and item length the item
+    // kernel reads and zeroes the completion counters, so what an earlier call
+    // left in the array needs no clearing here.
 
     // The profiler's CUDA events are created on demand; keep it out of this call.
     zha_profiler *prof = t->prof;
