@@ -8,13 +8,17 @@
 // with the same scale beta as the summaries:
 //   out = sum_i softmax_i(beta <q, k_i>) v_i,   lse = logsumexp_i(beta <q, k_i>).
 //
-// Design (split-K decode attention, fp32 accumulation, two launches):
-//   attend_plan   one CTA sums the walks' key counts, sets the item length from
-//                 that total so that the whole call has at most ITEM_BUDGET
-//                 items (never fewer than SEG_MIN keys each, never more than
-//                 MAX_SPLIT items per walk), and scans the walks' item and group
-//                 counts into offsets and an item -> walk map. Walks without
-//                 keys get out = 0, lse = -inf here.
+// Design (split-K decode attention, fp32 accumulation):
+//   plan          sum the walks' key counts, set the item length from that total
+//                 so that the whole call has at most ITEM_BUDGET items (never
+//                 fewer than SEG_MIN keys each, never more than MAX_SPLIT items
+//                 per walk), and scan the walks' item and group counts into
+//                 offsets. Walks without keys get out = 0, lse = -inf here. Calls
+//                 of up to LOCAL_MAX_W walks plan inside every CTA of
+//                 attend_items (shared memory; a warp finds its item's walk by
+//                 binary search) after a memset clears the completion counters;
+//                 larger calls run attend_plan (one CTA) first, which also writes
+//                 an item -> walk map and clears the counters.
 //   attend_items  grid-stride over items, one warp per item. The item's chunk
 //                 ids come through a two-window register prefetch (32 ids per
 //                 window, one per lane) and are broadcast by shuffle. A row of K
@@ -40,6 +44,7 @@ constexpr int SEG_MIN = 128;         // keys per work item, at least
 constexpr int MAX_SPLIT = 512;       // work items per walk, at most
 constexpr int ITEM_BUDGET = 16384;   // work items per call (before per-walk rounding)
 constexpr int GROUP = 16;            // items merged together first
+constexpr int LOCAL_MAX_W = 2048;    // calls of at most this many walks plan inside the item kernel
 
 __device__ __forceinline__ long long walk_keys(const int *sel_count, long long w, int max_sel, int C,
                                                long long tail) {
@@ -171,7 +176,7 @@ struct ItemArgs {
     int q_bf16, out_bf16;
     const int *sel, *sel_count, *item_off, *group_off, *seg, *item_walk;
     int *walk_done, *group_done;
-    int max_sel, C, G;
+    int max_sel, C, G, D;
     int c_shift;  // log2(C) when C is a power of two, else -1
     long long W, cap, n1, tail;
     float beta;
@@ -283,7 +288,72 @@ __device__ __forceinline__ void write_out(const ItemArgs &a, long long walk, int
     if (lane == 0 && a.lse) a.lse[walk] = empty ? -INFINITY : m + logf(l);
 }
 
-template <typename T, int D>
+// The plan of attend_plan_kernel, computed by one CTA into shared memory: item
+// offsets s_io[W + 1], group offsets s_go[W + 1] and key counts s_L[W] of every
+// walk; returns the call's item length. Walks without keys get out = 0,
+// lse = -inf from CTA 0. Used when the walks are few enough for every CTA to
+// plan for itself (the counts are a few KB, read from L2).
+__device__ long long local_plan(const ItemArgs &a, int *s_io, int *s_go, int *s_L) {
+    __shared__ long long sh[64];
+    const int W = (int)a.W, tid = threadIdx.x, nt = blockDim.x;
+    const int per = (W + nt - 1) / nt, w0 = min(W, tid * per), w1 = min(W, w0 + per);
+    long long keys = 0;
+    for (int w = w0; w < w1; ++w) {
+        const long long L = walk_keys(a.sel_count, w, a.max_sel, a.C, a.tail);
+        s_L[w] = (int)L;
+        keys += L;
+    }
+    long long zero = 0, total_keys, unused;
+    block_scan2(keys, zero, sh, total_keys, unused);
+    long long seg = (total_keys + ITEM_BUDGET - 1) / ITEM_BUDGET;
+    if (seg < SEG_MIN) seg = SEG_MIN;
+    if (seg > (1LL << 30)) seg = 1LL << 30;
+    long long ni = 0, ng = 0;
+    for (int w = w0; w < w1; ++w) {
+        const long long L = s_L[w], sw = seg_len(L, seg);
+        const long long items = L > 0 ? (L + sw - 1) / sw : 0;
+        ni += items;
+        ng += (items + GROUP - 1) / GROUP;
+    }
+    long long ii = ni, gi = ng, ti, tg;
+    block_scan2(ii, gi, sh, ti, tg);
+    ii -= ni;
+    gi -= ng;
+    for (int w = w0; w < w1; ++w) {
+        const long long L = s_L[w], sw = seg_len(L, seg);
+        const long long items = L > 0 ? (L + sw - 1) / sw : 0;
+        s_io[w] = (int)ii;
+        s_go[w] = (int)gi;
+        ii += items;
+        gi += (items + GROUP - 1) / GROUP;
+        if (items == 0 && blockIdx.x == 0) {
+            for (int e = 0; e < a.D; ++e) {
+                if (a.out_bf16) store_out(static_cast<__nv_bfloat16 *>(a.out) + (long long)w * a.D + e, 0.f);
+                else store_out(static_cast<float *>(a.out) + (long long)w * a.D + e, 0.f);
+            }
+            if (a.lse) a.lse[w] = -INFINITY;
+        }
+    }
+    if (tid == 0) {
+        s_io[W] = (int)ti;
+        s_go[W] = (int)tg;
+    }
+    __syncthreads();
+    return seg;
+}
+
+// Walk owning `item`: the last w with s_io[w] <= item (s_io[0] = 0 <= item < s_io[W]).
+__device__ __forceinline__ int find_walk(const int *s_io, int W, long long item) {
+    int lo = 0, hi = W;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_io[mid] <= item) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
+template <typename T, int D, bool LOCAL>
 __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
     constexpr int EPL = Row<T>::EPL;
     constexpr int LPR0 = D / EPL;
@@ -301,17 +371,27 @@ __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
     const int grp = lane / LPR, gl = lane % LPR;
     const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
-    const long long total = a.item_off[a.W];
-    const long long seg = a.seg[0];
+    extern __shared__ int s_plan[];  // LOCAL: item offsets [W + 1], group offsets [W + 1], keys [W]
+    const int *item_off = a.item_off, *group_off = a.group_off;
+    const int *s_L = s_plan + 2 * (a.W + 1);
+    long long seg;
+    if constexpr (LOCAL) {
+        seg = local_plan(a, s_plan, s_plan + (a.W + 1), s_plan + 2 * (a.W + 1));
+        item_off = s_plan;
+        group_off = s_plan + (a.W + 1);
+    } else {
+        seg = a.seg[0];
+    }
+    const long long total = item_off[a.W];
     const T *Kb = static_cast<const T *>(a.K);
     const T *Vb = static_cast<const T *>(a.V);
 
     for (long long item = gw; item < total; item += nw) {
-        const long long walk = a.item_walk[item];
+        const long long walk = LOCAL ? find_walk(item_off, (int)a.W, item) : a.item_walk[item];
         const long long tree = walk / a.G;
-        const long long L = walk_keys(a.sel_count, walk, a.max_sel, a.C, a.tail);
-        const long long i_first = a.item_off[walk];
-        const int nitems = a.item_off[walk + 1] - (int)i_first;
+        const long long L = LOCAL ? (long long)s_L[walk] : walk_keys(a.sel_count, walk, a.max_sel, a.C, a.tail);
+        const long long i_first = item_off[walk];
+        const int nitems = item_off[walk + 1] - (int)i_first;
         const long long sw = seg_len(L, seg);
         const long long k0 = (item - i_first) * sw;
         const long long k1 = k0 + sw < L ? k0 + sw : L;
@@ -474,8 +554,8 @@ __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
         __syncwarp();
         const int j = (int)(item - i_first), g = j / GROUP;
         const int gsize = nitems - g * GROUP < GROUP ? nitems - g * GROUP : GROUP;
-        const long long g_first = a.group_off[walk];
-        const int ngroups = a.group_off[walk + 1] - (int)g_first;
+        const long long g_first = group_off[walk];
+        const int ngroups = group_off[walk + 1] - (int)g_first;
         int ticket = 0;
         if (lane == 0) ticket = atomicAdd(a.group_done + g_first + g, 1) + 1;
         ticket = __shfl_sync(FULL, ticket, 0);
@@ -505,11 +585,13 @@ __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
     }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool LOCAL>
 cudaError_t launch_items(const zha_tree *t, const ItemArgs &ia, long long max_items, cudaStream_t st) {
     static int per_sm = 0;
+    const size_t smem = LOCAL ? sizeof(int) * (3 * (size_t)ia.W + 2) : 0;
     if (!per_sm) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attend_items_kernel<T, D>, 256, 0) != cudaSuccess ||
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attend_items_kernel<T, D, LOCAL>, 256,
+                                                          sizeof(int) * (3 * LOCAL_MAX_W + 2)) != cudaSuccess ||
             per_sm < 1)
             per_sm = 1;
     }
@@ -518,8 +600,14 @@ cudaError_t launch_items(const zha_tree *t, const ItemArgs &ia, long long max_it
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     Probe pr(t, ZHA_K_ATTEND_PARTIAL, st);
-    attend_items_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(ia);
+    attend_items_kernel<T, D, LOCAL><<<(unsigned)blocks, 256, smem, st>>>(ia);
     return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_items_any(const zha_tree *t, const ItemArgs &ia, long long max_items, cudaStream_t st) {
+    return ia.W <= LOCAL_MAX_W ? launch_items<T, D, true>(t, ia, max_items, st)
+                               : launch_items<T, D, false>(t, ia, max_items, st);
 }
 
 }  // namespace
@@ -559,6 +647,7 @@ void attend_carve(const AttendLayout &L, void *base, Scratch *s) {
     s->partial = reinterpret_cast<float *>(b + L.partial);
     s->gpartial = reinterpret_cast<float *>(b + L.gpartial);
     s->max_items = L.max_items;
+    s->max_groups = L.max_groups;
 }
 
 cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zha_dtype q_dtype, int G,
@@ -581,7 +670,14 @@ cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zh
     pl.group_done = s.group_done;
     pl.out = out;
     pl.lse = lse;
-    {
+    if (W <= LOCAL_MAX_W) {
+        // the item kernel plans for itself; only the completion counters (walk
+        // and group tickets, adjacent in the scratch) must start at zero
+        const size_t bytes = reinterpret_cast<const char *>(s.group_done + s.max_groups) -
+                             reinterpret_cast<const char *>(s.walk_done);
+        cudaError_t e = cudaMemsetAsync(s.walk_done, 0, bytes, st);
+        if (e != cudaSuccess) return e;
+    } else {
         Probe pr(t, ZHA_K_ATTEND_PLAN, st);
         attend_plan_kernel<<<1, 1024, 0, st>>>(pl);
         cudaError_t e = cudaGetLastError();
@@ -604,6 +700,7 @@ cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zh
     ia.group_done = s.group_done;
     ia.max_sel = max_sel;
     ia.C = c.chunk;
+    ia.D = c.d;
     ia.c_shift = (c.chunk & (c.chunk - 1)) == 0 ? __builtin_ctz((unsigned)c.chunk) : -1;
     ia.G = G;
     ia.W = W;
@@ -619,14 +716,14 @@ cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zh
     const bool bf = c.kv_dtype == ZHA_BF16;
     switch (c.d) {
         case 64:
-            return bf ? launch_items<__nv_bfloat16, 64>(t, ia, s.max_items, st)
-                      : launch_items<float, 64>(t, ia, s.max_items, st);
+            return bf ? launch_items_any<__nv_bfloat16, 64>(t, ia, s.max_items, st)
+                      : launch_items_any<float, 64>(t, ia, s.max_items, st);
         case 128:
-            return bf ? launch_items<__nv_bfloat16, 128>(t, ia, s.max_items, st)
-                      : launch_items<float, 128>(t, ia, s.max_items, st);
+            return bf ? launch_items_any<__nv_bfloat16, 128>(t, ia, s.max_items, st)
+                      : launch_items_any<float, 128>(t, ia, s.max_items, st);
         default:
-            return bf ? launch_items<__nv_bfloat16, 256>(t, ia, s.max_items, st)
-                      : launch_items<float, 256>(t, ia, s.max_items, st);
+            return bf ? launch_items_any<__nv_bfloat16, 256>(t, ia, s.max_items, st)
+                      : launch_items_any<float, 256>(t, ia, s.max_items, st);
     }
 }
 

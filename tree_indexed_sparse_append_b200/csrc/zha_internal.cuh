@@ -212,7 +212,7 @@ struct Scratch {
     int *group_done;           // [max_groups] attend items finished per group
     float *partial;            // [max_items][D + 4]
     float *gpartial;           // [max_groups][D + 4]
-    long long Sstride, Lstride, max_items;
+    long long Sstride, Lstride, max_items, max_groups;
 };
 
 int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s);
