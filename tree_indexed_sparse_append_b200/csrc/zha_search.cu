@@ -316,18 +316,20 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t x, unsigned *sh) {
 // Each walk's frontier keys are staged once, in shared memory when they fit
 // (smem_keys), else in the walk's row of a global key array. The cutoff is found
 // with at most three kinds of histogram pass, each over 256 buckets that keep
-// count, fixed-point mass and largest key (HCOPIES copies, shared by groups of
-// warps):
+// count and fixed-point mass (HCOPIES copies, shared by groups of warps):
 //   1. coarse: 1/8 nat per bucket below the frontier's highest score (keys
 //      spread over many buckets, so the atomics rarely collide; this pass also
 //      yields the total mass);
 //   2. fine: 1/2048 nat inside the crossing coarse bucket;
 //   3. radix on the raw score bits inside the crossing fine bucket, a byte at a
-//      time (only when several keys share that 1/2048-nat bucket).
+//      time.
 // Bucket orders agree with the score order, so the crossing bucket of each pass
-// holds the cutoff; a bucket with a single key ends the search.
+// holds the cutoff. As soon as it holds at most CAND_MAX keys, they are listed
+// and one warp ranks them directly (mass strictly above each, mass of its equal
+// keys), which ends the search.
 constexpr int HCOPIES = 8;
 constexpr float COARSE_PER_NAT = 8.f;
+constexpr int CAND_MAX = 32;  // a crossing bucket this small is resolved by one warp
 
 __device__ __forceinline__ int coarse_bucket(float s, float m) {
     const float x = (m - s) * COARSE_PER_NAT;
@@ -343,13 +345,13 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
     extern __shared__ uint32_t skey_s[];
     __shared__ unsigned long long h_mass[HCOPIES][256];
     __shared__ unsigned h_cnt[HCOPIES][256];
-    __shared__ unsigned h_max[HCOPIES][256];
     __shared__ unsigned long long sh_u64[NT / 32];
     __shared__ unsigned sh_u32[NT / 32];
+    __shared__ uint32_t s_cand[CAND_MAX];
     __shared__ int s_bucket;
     __shared__ uint32_t s_key;
     __shared__ unsigned long long s_trem;
-    __shared__ unsigned s_krem, s_count;
+    __shared__ unsigned s_krem, s_count, s_ncand;
 
     const long long walk = blockIdx.x;
     const int tid = threadIdx.x;
@@ -401,32 +403,30 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
         // stage 0: coarse, 1: fine, 2..5: raw bytes 24, 16, 8, 0
         int cb = -1, fb = -1;
         uint32_t prefix = 0, pmask = 0;
+        // keys still in play after `narrowed` stages: the crossing buckets so far
+        auto in_play = [&](uint32_t k, int narrowed) -> bool {
+            if (narrowed == 0) return true;
+            const float s = key_to_float(k);
+            if (coarse_bucket(s, m) != cb) return false;
+            if (narrowed == 1) return true;
+            return fine_bucket(s, m, cb) == fb && (k & pmask) == prefix;
+        };
         bool done = false;
         for (int stage = 0; stage < 6 && !done; ++stage) {
             for (int j = tid; j < HCOPIES * 256; j += NT) {
                 (&h_mass[0][0])[j] = 0;
                 (&h_cnt[0][0])[j] = 0;
-                (&h_max[0][0])[j] = 0;
             }
+            if (tid == 0) s_ncand = 0;
             __syncthreads();
             const int shift = 24 - 8 * (stage - 2);
             for (long long i = tid; i < F; i += NT) {
                 const uint32_t k = key_at(i);
+                if (!in_play(k, stage)) continue;
                 const float s = key_to_float(k);
-                int b;
-                if (stage == 0) {
-                    b = coarse_bucket(s, m);
-                } else {
-                    if (coarse_bucket(s, m) != cb) continue;
-                    if (stage == 1) {
-                        b = fine_bucket(s, m, cb);
-                    } else {
-                        if (fine_bucket(s, m, cb) != fb || (k & pmask) != prefix) continue;
-                        b = (k >> shift) & 255;
-                    }
-                }
+                const int b = stage == 0 ? coarse_bucket(s, m)
+                                         : (stage == 1 ? fine_bucket(s, m, cb) : (int)((k >> shift) & 255));
                 atomicAdd(&h_cnt[wcopy][b], 1u);
-                atomicMax(&h_max[wcopy][b], k);
                 if (top_p) atomicAdd(&h_mass[wcopy][b], mass(s));
             }
             __syncthreads();
@@ -436,13 +436,12 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
             const bool own = tid < 256;
             const int b = own ? (stage >= 2 ? 255 - tid : tid) : 0;
             unsigned long long vm = 0;
-            unsigned vc = 0, vx = 0;
+            unsigned vc = 0;
             if (own) {
 #pragma unroll
                 for (int c = 0; c < HCOPIES; ++c) {
                     vm += h_mass[c][b];
                     vc += h_cnt[c][b];
-                    vx = max(vx, h_max[c][b]);
                 }
             }
             unsigned long long total_m;
@@ -457,7 +456,6 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
                                            : (incl_c - vc < krem && krem <= incl_c));
             if (hit) {
                 s_bucket = b;
-                s_key = vx;
                 s_trem = trem - (incl_m - vm);
                 s_krem = krem - (incl_c - vc);
                 s_count = vc;
@@ -466,21 +464,71 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
             const int hb = s_bucket;
             trem = s_trem;
             krem = s_krem;
-            eq_count = s_count;
-            if (eq_count == 1) {
-                kstar = s_key;
-                done = true;
-            } else if (stage == 0) {
+            const unsigned cnt = s_count;
+            if (stage == 0) {
                 cb = hb;
             } else if (stage == 1) {
                 fb = hb;
             } else {
                 prefix |= (uint32_t)hb << shift;
                 pmask |= 255u << shift;
-                if (stage == 5) {
-                    kstar = prefix;
-                    done = true;
+            }
+            if (cnt <= CAND_MAX) {
+                // few keys left: list them and let one warp rank them directly
+                for (long long i = tid; i < F; i += NT) {
+                    const uint32_t k = key_at(i);
+                    if (in_play(k, stage + 1)) {
+                        const unsigned slot = atomicAdd(&s_ncand, 1u);
+                        if (slot < CAND_MAX) s_cand[slot] = k;
+                    }
                 }
+                __syncthreads();
+                if (tid < 32) {
+                    const int lane = tid;
+                    const int n = min(s_ncand, (unsigned)CAND_MAX);
+                    const bool v = lane < n;
+                    const uint32_t kj = v ? s_cand[lane] : 0u;
+                    const unsigned long long uj = v ? (top_p ? mass(key_to_float(kj)) : 1ull) : 0ull;
+                    unsigned long long above = 0, same = 0;
+                    unsigned same_n = 0;
+#pragma unroll
+                    for (int i = 0; i < CAND_MAX; ++i) {
+                        const uint32_t ki = __shfl_sync(FULL, kj, i);
+                        const unsigned long long ui = __shfl_sync(FULL, uj, i);
+                        if (i < n) {
+                            if (ki > kj) above += ui;
+                            else if (ki == kj) {
+                                same += ui;
+                                ++same_n;
+                            }
+                        }
+                    }
+                    const unsigned long long target = top_p ? trem : (unsigned long long)krem;
+                    unsigned bal = __ballot_sync(FULL, v && above < target && target <= above + same);
+                    if (!bal) {  // cannot happen while the sums agree; then open the whole bucket
+                        uint32_t kmin = v ? kj : 0xffffffffu;
+#pragma unroll
+                        for (int o = 16; o >= 1; o >>= 1) kmin = min(kmin, __shfl_xor_sync(FULL, kmin, o));
+                        bal = __ballot_sync(FULL, v && kj == kmin);
+                    }
+                    const int src = bal ? __ffs(bal) - 1 : 0;
+                    if (lane == src) {
+                        s_key = kj;
+                        s_trem = trem - above;
+                        s_krem = krem - (unsigned)above;
+                        s_count = same_n;
+                    }
+                }
+                __syncthreads();
+                kstar = s_key;
+                trem = s_trem;
+                krem = s_krem;
+                eq_count = s_count;
+                done = true;
+            } else if (stage == 5) {
+                kstar = prefix;  // every key left equals prefix
+                eq_count = cnt;
+                done = true;
             }
             __syncthreads();
         }
@@ -546,22 +594,34 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
         unsigned *M_tree = a.M_next ? a.M_next + (long long)t * a.words_next * a.G : nullptr;
         unsigned *U_tree = a.U_next ? a.U_next + (long long)t * a.words_next : nullptr;
         unsigned eq = eq_base, eqg, rank = open_base;
-        for (long long i0 = rbeg; i0 < rend; i0 += 32) {
-            const long long i = i0 + lane;
-            const bool o = opened(i, eq, eqg);
-            const unsigned om = __ballot_sync(FULL, o);
-            if (o) {
-                const unsigned r = rank + __popc(om & below);
-                const long long id = frontier_id(a, par, npar, i);
-                if (a.level == 1) {
-                    if (r < (unsigned)a.max_sel) a.sel[walk * a.max_sel + r] = (int)id;
-                } else {
-                    a.par_out[walk * a.Lstride + r] = (int)id;
-                    set_bits(M_tree, U_tree, a.G, g, id * a.C, id * a.C + a.C);
-                }
+        // node ids of 8 groups of 32 positions are loaded before any is used
+        for (long long i00 = rbeg; i00 < rend; i00 += 32 * 8) {
+            long long idv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const long long i = i00 + 32 * u + lane;
+                idv[u] = i < rend ? frontier_id(a, par, npar, i) : 0;
             }
-            rank += __popc(om);
-            eq += eqg;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const long long i0 = i00 + 32 * u;
+                if (i0 >= rend) break;
+                const long long i = i0 + lane;
+                const bool o = opened(i, eq, eqg);
+                const unsigned om = __ballot_sync(FULL, o);
+                if (o) {
+                    const unsigned r = rank + __popc(om & below);
+                    const long long id = idv[u];
+                    if (a.level == 1) {
+                        if (r < (unsigned)a.max_sel) a.sel[walk * a.max_sel + r] = (int)id;
+                    } else {
+                        a.par_out[walk * a.Lstride + r] = (int)id;
+                        set_bits(M_tree, U_tree, a.G, g, id * a.C, id * a.C + a.C);
+                    }
+                }
+                rank += __popc(om);
+                eq += eqg;
+            }
         }
         if (a.level > 1 && a.n_orph_next > 0) {
             const long long lo = a.n_level_next - a.n_orph_next, hi = a.n_level_next;
