@@ -397,6 +397,61 @@ def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes
             "n_keys_after": n_after, "dense": dense}
 
 
+def run_prefill(args, dev):
+    """Search + attend of the prefill workload (4,096 queries per query head against
+    one sequence's 262,144-key trees), timed on the device; no append."""
+    import torch
+
+    import synthetic as S
+    import tree_indexed_sparse_append_b200 as Z
+
+    w = S.WORKLOADS["prefill256k"]
+    inp = S.draw(w, device="cuda")
+    st = torch.cuda.current_stream()
+    tree = Z.Tree(inp.K, inp.V, inp.refs, w.n_keys, w.chunk, w.depth, w.beta, w.top_width)
+    Wk = w.walks
+    max_sel = tree.level(1)[1]
+    sel = torch.empty(Wk, max_sel, dtype=torch.int32, device=dev)
+    cnt = torch.empty(Wk, dtype=torch.int32, device=dev)
+    out = torch.empty_like(inp.Q, dtype=inp.K.dtype)
+    lse = torch.empty(Wk, dtype=torch.float32, device=dev)
+    tree.reserve(Wk, max_sel)
+
+    def step():
+        tree.search(inp.Q, Z.TOP_P, 0.9, 0, max_sel=max_sel, out=(sel, cnt, None))
+        tree.attend(inp.Q, sel, cnt, out=out, lse=lse)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        step()
+        e1.record(st)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ms = sorted(ts)[len(ts) // 2]
+    tree.profile(True)
+    step()
+    info = tree.last_search_info()
+    kt = {k: round(v[1], 4) for k, v in tree.profile_read().items() if v[0]}
+    tree.profile(False)
+    tree.sync_status()
+    walk_nodes = sum(info["walk_nodes"][1:info["start_level"] + 1])
+    flops = 2.0 * w.R * w.d * walk_nodes
+    res = {"workload": "prefill: 4,096 queries x 16 q-heads against the 4 KV-head trees of one 262,144-key "
+                       "sequence, d=128, bf16, C=8, depth 6, R=8, top-p 0.9",
+           "walks": Wk, "ms": ms, "value": Wk / (ms / 1e3), "unit": UNIT, "kernel_ms": kt,
+           "score_tflops": flops / (kt["score"] / 1e3) / 1e12 if kt.get("score") else None,
+           "scored_walk_nodes": walk_nodes, "union_nodes": sum(info["union_nodes"][1:info["start_level"] + 1])}
+    tree.close()
+    del inp, sel, cnt, out, lse
+    torch.cuda.empty_cache()
+    return res
+
+
 def config_of(w, label):
     return {"workload": label, "sequences": w.batch, "kv_heads": w.n_kv_heads, "q_heads": w.n_q_heads,
             "keys": w.n_keys, "d": w.d, "kv_dtype": w.kv_dtype, "chunk": w.chunk, "depth": w.depth, "R": w.R,
@@ -439,6 +494,9 @@ def main():
                                "kernel_ms_per_step": r["kernel_ms_per_step"], "clocks": r["clocks"]}
                            for m, r in x["results"].items()},
                  "e2e": x["e2e"], "dense_scan": x["dense"]}
+    prefill = None
+    if not args.no_extra and rank == 0:
+        prefill = run_prefill(args, dev)
     r = head["results"]["top_p"]
     line = {
         "metric": METRIC, "value": r["qps"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -450,6 +508,7 @@ def main():
         "clocks": r["clocks"], "kernel_ms_per_step": r["kernel_ms_per_step"],
         "build": {"ms": head["build_ms"], "keys_per_s": head["w"].trees * head["w"].n_keys / (head["build_ms"] / 1e3)},
         "kv1m": extra,
+        "prefill": prefill,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -1,0 +1,99 @@
+"""Tensor-core scoring (trees walked by at least 1,024 bf16 queries): parity with
+the oracle, and agreement with the CUDA-core scorer on the same query values.
+
+The workload: one sequence, 2 KV heads and 4 query heads (2:1), 550 queries per
+query head, so 1,100 walks per tree (not a multiple of the 128-walk tile); 16,427
+clustered keys (blocks of 64 around random centres) with C = 8 and depth 4, so
+level sizes 2,053 / 256 / 32 / 4 and a ragged tail of 3 keys; R = 6 reference
+queries (padded to 8 columns per node); d = 128, bf16 keys, values and queries.
+Every level the walk visits is scored on the tensor cores.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from helpers import assert_attention_close, compare_selection, host64, near_tie
+
+pytestmark = pytest.mark.gpu
+
+N, C, DEPTH, D, R, H, HQ, NQ = 16427, 8, 4, 128, 6, 2, 4, 550
+BETA = 1 / np.sqrt(D)
+
+
+def zha():
+    import tree_indexed_sparse_append_b200 as Z
+
+    return Z
+
+
+def inputs(seed=7):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    blocks = (N + 63) // 64
+    centres = torch.randn(H, blocks, D, generator=g, device="cuda")
+    K = (centres.repeat_interleave(64, dim=1)[:, :N] + 0.3 * torch.randn(H, N, D, generator=g, device="cuda"))
+    V = torch.randn(H, N, D, generator=g, device="cuda")
+    refs = torch.randn(H, R, D, generator=g, device="cuda")
+    # queries: the sum of 1 to 3 centres of their tree
+    Q = torch.zeros(HQ, NQ, D, device="cuda")
+    group = HQ // H
+    for hq in range(HQ):
+        m = torch.randint(1, 4, (NQ,), generator=g, device="cuda")
+        for j in range(3):
+            pick = torch.randint(0, blocks, (NQ,), generator=g, device="cuda")
+            Q[hq] += centres[hq // group, pick] * (m > j).unsqueeze(1)
+    return (K.to(torch.bfloat16)[None], V.to(torch.bfloat16)[None], refs, Q.to(torch.bfloat16)[None])
+
+
+def sample_walks():
+    # walks at the edges of the 128-walk tiles and spread over each tree
+    G = (HQ // H) * NQ
+    picks = set()
+    for t in range(H):
+        for r in list(range(0, G, 37)) + [0, 127, 128, 255, 256, 1023, 1024, G - 1]:
+            if r < G:
+                picks.add(t * G + r)
+    return sorted(picks)
+
+
+@pytest.mark.parametrize("mode,p,k", [(O.TOP_P, 0.9, 0), (O.TOP_K, 0, 8)])
+def test_tensor_core_search_matches_oracle(mode, p, k):
+    Z = zha()
+    K, V, refs, Q = inputs()
+    tree = Z.Tree(K, V, refs, N, C, DEPTH, BETA)
+    max_sel = N // C
+    sel, cnt, st = tree.search(Q, mode, p, k, max_sel=max_sel, with_stats=True)
+    out, lse = tree.attend(Q, sel, cnt, out_dtype=torch.float32)
+    tree.sync_status()
+    sel_h, cnt_h = sel.cpu().numpy(), cnt.cpu().numpy()
+    stats = Z.parse_stats(st)
+    out = host64(out).reshape(-1, D)
+    lse = lse.cpu().numpy()
+    Qh = host64(Q).reshape(-1, D)
+    G = (HQ // H) * NQ
+    otrees = [O.build_tree(host64(K[0, h, :N]), host64(refs[h]), C, DEPTH, BETA, store=O.STORE_F32) for h in range(H)]
+    checked = 0
+    for wi in sample_walks():
+        h = wi // G
+        ow = O.search(otrees[h], Qh[wi], mode, p, k, 64)
+        if compare_selection(sel_h, cnt_h, {wi: ow}):
+            continue
+        assert stats[wi]["work"] == ow.work and stats[wi]["keys_read"] == ow.keys_read
+        o_out, o_lse = O.attend(host64(K[0, h, :N]), host64(V[0, h, :N]), Qh[wi], ow.sel, C,
+                                otrees[h].n_nodes[1], BETA)
+        assert_attention_close(out[wi], lse[wi], o_out, o_lse, 3e-3, f"walk {wi}")
+        checked += 1
+    assert checked > 0.9 * len(sample_walks())
+
+    # the same query values as fp32 take the CUDA-core scorer
+    sel2, cnt2, _ = tree.search(Q.float(), mode, p, k, max_sel=max_sel)
+    tree.sync_status()
+    sel2, cnt2 = sel2.cpu().numpy(), cnt2.cpu().numpy()
+    differ = [w for w in range(sel_h.shape[0])
+              if cnt_h[w] != cnt2[w] or not np.array_equal(sel_h[w, :cnt_h[w]], sel2[w, :cnt2[w]])]
+    for wi in differ:
+        ow = O.search(otrees[wi // G], Qh[wi], mode, p, k, 64)
+        assert near_tie(ow), f"walk {wi}: tensor-core and CUDA-core selections differ away from a tie"
+    print(f"tensor-core scoring: {checked} sampled walks match the oracle; "
+          f"{len(differ)} of {sel_h.shape[0]} walks part from the CUDA-core path, all at oracle near-ties")
+    tree.close()

@@ -164,6 +164,15 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     const size_t U_bytes = off - U_start;
     const AttendLayout att = attend_layout(W, c.d);
     const size_t o_att = take(att.bytes);
+    // tensor-core scoring tiles, for trees walked by many queries
+    const long long Gw = W / t->T;
+    size_t tc_bytes = 0;
+    if (c.d == 128 && Gw >= TC_MIN_G) {
+        long long maxn = 0;
+        for (int l = 1; l <= c.depth; ++l) maxn = std::max(maxn, std::min(t->cap_nodes[l], TC_MAX_NODES));
+        if (maxn > 0) tc_bytes = tc_scratch_bytes(t->T, Gw, maxn, c.R);
+    }
+    const size_t o_tc = take(tc_bytes);
     const size_t need = off;
 
     if (need > t->ws_bytes) {
@@ -194,6 +203,7 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     s->M_bytes = M_bytes;
     s->U_bytes = U_bytes;
     attend_carve(att, b + o_att, s);
+    s->tc = tc_bytes ? reinterpret_cast<unsigned char *>(b + o_tc) : nullptr;
     s->Sstride = cap1;
     s->Lstride = cap2;
     return ZHA_OK;
@@ -417,6 +427,7 @@ int zha_sync_status(zha_tree *t, void *stream) {
     ZHA_CUDA(cudaMemset(t->d_status, 0, sizeof(int)), "clearing the status word");
     if (code == zha::DEV_CAPACITY) return fail(ZHA_ERR_CAPACITY, "a walk opened more level-1 nodes than max_sel");
     if (code == zha::DEV_BAD_INDEX) return fail(ZHA_ERR_INTERNAL, "a selected chunk id was out of range");
+    if (code == zha::DEV_TIMEOUT) return fail(ZHA_ERR_TIMEOUT, "a bounded wait inside a kernel gave up");
     if (code) return fail(ZHA_ERR_INTERNAL, "device status %d", code);
     return ZHA_OK;
 }

@@ -13,7 +13,7 @@ namespace zha {
 constexpr unsigned FULL = 0xffffffffu;
 
 // Device-side error codes recorded in the tree's status word (first one wins).
-enum : int { DEV_OK = 0, DEV_CAPACITY = 1, DEV_BAD_INDEX = 2 };
+enum : int { DEV_OK = 0, DEV_CAPACITY = 1, DEV_BAD_INDEX = 2, DEV_TIMEOUT = 3 };
 
 __device__ __forceinline__ void report(int *status, int code) {
     if (status) atomicCAS(status, DEV_OK, code);
@@ -212,6 +212,7 @@ struct Scratch {
     int *group_done;           // [max_groups] attend items finished per group
     float *partial;            // [max_items][D + 4]
     float *gpartial;           // [max_groups][D + 4]
+    unsigned char *tc;         // tensor-core scoring tiles (NULL when the walks per tree are few)
     long long Sstride, Lstride, max_items, max_groups;
 };
 
@@ -226,6 +227,17 @@ struct AttendLayout {
 AttendLayout attend_layout(long long W, int D);
 // Points the attention fields of s into the block at base laid out by L.
 void attend_carve(const AttendLayout &L, void *base, Scratch *s);
+
+// Tensor-core scoring of a whole level (zha_score_tc.cu), used for trees of at
+// least TC_MIN_G walks, levels of at most TC_MAX_NODES nodes, d = 128 and bf16
+// queries; other calls score on the CUDA cores.
+constexpr int TC_MIN_G = 1024;
+constexpr long long TC_MAX_NODES = 8192;
+size_t tc_scratch_bytes(int T, long long G, long long max_level_nodes, int R);
+bool tc_applicable(const zha_tree *t, int G, const void *Q, zha_dtype q_dtype, int level);
+cudaError_t launch_score_tc_queries(const zha_tree *t, const void *Q, int G, unsigned char *ws, cudaStream_t st);
+cudaError_t launch_score_tc(const zha_tree *t, int level, int G, unsigned char *ws, float *S, long long Sstride,
+                            cudaStream_t st);
 // Records an error message for zha_last_error (this host thread); returns code.
 int set_error(int code, const char *msg);
 

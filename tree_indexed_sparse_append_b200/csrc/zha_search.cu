@@ -774,30 +774,44 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
 
+    // trees walked by many bf16 queries score whole small levels on the tensor cores
+    bool tc_any = false;
+    if (s.tc)
+        for (int l = start_level; l >= 1; --l) tc_any = tc_any || tc_applicable(t, G, Q, q_dtype, l);
+    if (tc_any) {
+        e = launch_score_tc_queries(t, Q, G, s.tc, st);
+        if (e != cudaSuccess) return e;
+    }
+
     int cur = 0;
     for (int l = start_level; l >= 1; --l) {
-        ScoreArgs sa{};
-        sa.nodes = t->nodes[l];
-        sa.node_tree = t->cap_nodes[l] * t->NF;
-        sa.NF = t->NF;
-        sa.R = c.R;
-        sa.G = G;
-        sa.T = t->T;
-        sa.beta = c.sharpness;
-        sa.U = s.U[l];
-        sa.M = s.M[l];
-        sa.words = words(l);
-        sa.n_level = t->n_nodes[l];
-        sa.qf = s.qf;
-        sa.S = s.S;
-        sa.Sstride = s.Sstride;
-        sa.npi = 4;
-        switch (D) {
-            case 64: e = launch_score_d<64>(t, sa, st); break;
-            case 128: e = launch_score_d<128>(t, sa, st); break;
-            default: e = launch_score_d<256>(t, sa, st); break;
+        if (tc_any && tc_applicable(t, G, Q, q_dtype, l)) {
+            e = launch_score_tc(t, l, G, s.tc, s.S, s.Sstride, st);
+            if (e != cudaSuccess) return e;
+        } else {
+            ScoreArgs sa{};
+            sa.nodes = t->nodes[l];
+            sa.node_tree = t->cap_nodes[l] * t->NF;
+            sa.NF = t->NF;
+            sa.R = c.R;
+            sa.G = G;
+            sa.T = t->T;
+            sa.beta = c.sharpness;
+            sa.U = s.U[l];
+            sa.M = s.M[l];
+            sa.words = words(l);
+            sa.n_level = t->n_nodes[l];
+            sa.qf = s.qf;
+            sa.S = s.S;
+            sa.Sstride = s.Sstride;
+            sa.npi = 4;
+            switch (D) {
+                case 64: e = launch_score_d<64>(t, sa, st); break;
+                case 128: e = launch_score_d<128>(t, sa, st); break;
+                default: e = launch_score_d<256>(t, sa, st); break;
+            }
+            if (e != cudaSuccess) return e;
         }
-        if (e != cudaSuccess) return e;
 
         SelectArgs se{};
         se.level = l;
