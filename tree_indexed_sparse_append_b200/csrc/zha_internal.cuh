@@ -151,10 +151,10 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
 }
 
 // Frontier masses are summed as unsigned fixed point with 40 fractional bits:
-// the sums are exact and independent of the order of addition.
-constexpr double MASS_ONE = 1099511627776.0;  // 2^40
+// the sums are exact and independent of the order of addition. e * 2^40 is exact
+// in fp32 (a power-of-two scale), so converting it rounds that exact value.
 __device__ __forceinline__ unsigned long long mass_fixed(float e) {
-    return (unsigned long long)__double2ull_rn((double)e * MASS_ONE);
+    return __float2ull_rn(e * 1099511627776.0f);
 }
 
 }  // namespace zha

@@ -734,7 +734,7 @@ cudaError_t launch_select_all(const zha_tree *t, const float *S, uint32_t *gkey,
     Probe pr(t, ZHA_K_SELECT, st);
     if (N > 8192) {
         se.smem_keys = std::min<long long>(N, 16384);
-        return launch_select<512>(se, W, st);
+        return launch_select<1024>(se, W, st);
     }
     se.smem_keys = N;
     return launch_select<256>(se, W, st);
@@ -848,7 +848,7 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
             Probe pr(t, ZHA_K_SELECT, st);
             if (t->n_nodes[l] > 8192) {
                 se.smem_keys = std::min<long long>(t->n_nodes[l], 16384);
-                e = launch_select<512>(se, W, st);
+                e = launch_select<1024>(se, W, st);
             } else {
                 se.smem_keys = t->n_nodes[l];
                 e = launch_select<256>(se, W, st);
