@@ -49,6 +49,10 @@ def parse():
     ap.add_argument("--profile-steps", type=int, default=20)
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--batch", type=int, default=0, help="sequences per GPU (default: the workload's)")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time only the prefill workload and print its line (for profiling)")
+    ap.add_argument("--prefill-queries", type=int, default=0,
+                    help="queries per query head of the prefill workload (default: the workload's 4,096)")
     return ap.parse_args()
 
 
@@ -406,6 +410,8 @@ def run_prefill(args, dev):
     import tree_indexed_sparse_append_b200 as Z
 
     w = S.WORKLOADS["prefill256k"]
+    if getattr(args, "prefill_queries", 0):
+        w = S.scaled(w, queries_per_head=args.prefill_queries)
     inp = S.draw(w, device="cuda")
     st = torch.cuda.current_stream()
     tree = Z.Tree(inp.K, inp.V, inp.refs, w.n_keys, w.chunk, w.depth, w.beta, w.top_width)
@@ -441,8 +447,8 @@ def run_prefill(args, dev):
     tree.sync_status()
     walk_nodes = sum(info["walk_nodes"][1:info["start_level"] + 1])
     flops = 2.0 * w.R * w.d * walk_nodes
-    res = {"workload": "prefill: 4,096 queries x 16 q-heads against the 4 KV-head trees of one 262,144-key "
-                       "sequence, d=128, bf16, C=8, depth 6, R=8, top-p 0.9",
+    res = {"workload": f"prefill: {w.queries_per_head:,} queries x 16 q-heads against the 4 KV-head trees of one "
+                       "262,144-key sequence, d=128, bf16, C=8, depth 6, R=8, top-p 0.9",
            "walks": Wk, "ms": ms, "value": Wk / (ms / 1e3), "unit": UNIT, "kernel_ms": kt,
            "score_tflops": flops / (kt["score"] / 1e3) / 1e12 if kt.get("score") else None,
            "scored_walk_nodes": walk_nodes, "union_nodes": sum(info["union_nodes"][1:info["start_level"] + 1])}
@@ -472,6 +478,10 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", 0))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.prefill_only:
+        if rank == 0:
+            print(json.dumps(run_prefill(args, dev)), flush=True)
+        return
     if world > 1:
         import datetime
 

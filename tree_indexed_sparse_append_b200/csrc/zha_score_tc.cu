@@ -23,11 +23,13 @@
 //   tc_prep_queries  the tree's queries -> A tiles of 128 walks, same order.
 //   score_tc_kernel  one CTA per A tile: the A tile stays in shared memory, the B
 //                    tiles stream through a two-stage ring filled by bulk copies
-//                    (cp.async.bulk, no multicast), one thread issues the
-//                    tcgen05.mma (M = N = 128, K = 16, bf16 -> fp32 in TMEM) into
-//                    two accumulators used in turn, and four warps read a finished
-//                    accumulator back (tcgen05.ld), take the max over references
-//                    and store the scores.
+//                    (cp.async.bulk, no multicast; a stage is refilled as soon as
+//                    the MMAs reading it complete, the biases go to a ring of
+//                    their own), one thread issues the tcgen05.mma (M = N = 128,
+//                    K = 16, bf16 -> fp32 in TMEM) into two accumulators used in
+//                    turn, and four warps read a finished accumulator back
+//                    (tcgen05.ld), take the max over references and store the
+//                    scores.
 // Every wait is bounded: on timeout the kernel records DEV_TIMEOUT, waits (also
 // bounded) for its own copies and MMAs, frees its TMEM and returns.
 #include <cstdint>
@@ -44,7 +46,9 @@ constexpr int TC_PART = TC_N * TC_K * 2;             // bytes of one bf16 part o
 constexpr int TC_BTILE = 3 * TC_PART + TC_N * 4;     // hi, mid, lo, biases
 constexpr int TC_ATILE = TC_M * TC_K * 2;
 constexpr int TC_STAGES = 2;
-constexpr int TC_SMEM = TC_ATILE + TC_STAGES * TC_BTILE + 128;  // + barriers and the TMEM address
+constexpr int TC_BIAS_SLOTS = 4;                     // a tile's biases outlive its B stage
+constexpr int TC_STAGE = 3 * TC_PART;                // shared memory of one B stage (the three parts)
+constexpr int TC_SMEM = TC_ATILE + TC_STAGES * TC_STAGE + TC_BIAS_SLOTS * TC_N * 4 + 128;  // + barriers, TMEM address
 constexpr int TC_TMEM_COLS = 2 * TC_N;               // two fp32 accumulators of 128 columns
 constexpr unsigned long long TC_WAIT_NS = 1000000000ull;  // a wait gives up after 1 s
 
@@ -239,14 +243,15 @@ struct ScoreTcArgs {
 template <int RP>
 __global__ void __launch_bounds__(128, 1) score_tc_kernel(ScoreTcArgs a) {
     constexpr int NPT = TC_N / RP;  // nodes per B tile
-    extern __shared__ __align__(1024) unsigned char smem[];
+    extern __shared__ __align__(16) unsigned char smem[];  // no static shared memory: all of it is here
     unsigned char *sA = smem;
     unsigned char *sB = smem + TC_ATILE;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TC_ATILE + TC_STAGES * TC_BTILE);
+    float *sBias = reinterpret_cast<float *>(smem + TC_ATILE + TC_STAGES * TC_STAGE);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TC_ATILE + TC_STAGES * TC_STAGE + TC_BIAS_SLOTS * TC_N * 4);
     // bars[0..1]: B stage s filled (bulk copies); bars[2..3]: accumulator s written
     // (MMA commit); bars[4]: A tile filled
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
-    __shared__ int s_fail;
+    int &s_fail = *reinterpret_cast<int *>(bars + 7);
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const long long mt = blockIdx.x, t = blockIdx.y;
@@ -276,16 +281,20 @@ __global__ void __launch_bounds__(128, 1) score_tc_kernel(ScoreTcArgs a) {
     // bit 0: A copy; bits 1..2: B stage copies; bits 3..4: MMA groups
     unsigned pending = 0;
     long long issued_full[TC_STAGES] = {0, 0}, issued_mma[TC_STAGES] = {0, 0};  // uses so far, per barrier
+    // B tile n -> stage s: its three parts into the stage, its biases into slot n % 4
+    auto fill = [&](long long n, int s) {
+        const unsigned char *src = btree + n * TC_BTILE;
+        mbar_expect_tx(bar_full(s), TC_BTILE);
+        bulk_g2s(smem_u32(sB + s * TC_STAGE), src, TC_STAGE, bar_full(s));
+        bulk_g2s(smem_u32(sBias + (n & (TC_BIAS_SLOTS - 1)) * TC_N), src + TC_STAGE, TC_N * 4, bar_full(s));
+        pending |= 2u << s;
+        ++issued_full[s];
+    };
     if (tid == 0) {
         mbar_expect_tx(barA, TC_ATILE);
         bulk_g2s(smem_u32(sA), a.atiles + (t * a.mtiles + mt) * TC_ATILE, TC_ATILE, barA);
         pending |= 1u;
-        for (int s = 0; s < TC_STAGES && s < ntiles; ++s) {
-            mbar_expect_tx(bar_full(s), TC_BTILE);
-            bulk_g2s(smem_u32(sB + s * TC_BTILE), btree + (long long)s * TC_BTILE, TC_BTILE, bar_full(s));
-            pending |= 2u << s;
-            ++issued_full[s];
-        }
+        for (int s = 0; s < TC_STAGES && s < ntiles; ++s) fill(s, s);
     }
 
     const long long g = mt * TC_M + tid;  // this thread's walk within the tree (row of the tile)
@@ -305,7 +314,7 @@ __global__ void __launch_bounds__(128, 1) score_tc_kernel(ScoreTcArgs a) {
             }
         }
         tc_fence_after();
-        const float *bias = reinterpret_cast<const float *>(sB + s * TC_BTILE + 3 * TC_PART);
+        const float *bias = sBias + (n & (TC_BIAS_SLOTS - 1)) * TC_N;
         const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(s * TC_N);
         float sc[TC_N];
 #pragma unroll
@@ -354,7 +363,7 @@ __global__ void __launch_bounds__(128, 1) score_tc_kernel(ScoreTcArgs a) {
             } else {
                 pending &= ~(2u << s);
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB + s * TC_BTILE);
+                const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB + s * TC_STAGE);
                 const uint32_t d = tmem + (uint32_t)(s * TC_N);
 #pragma unroll
                 for (int part = 0; part < 3; ++part)
@@ -365,6 +374,17 @@ __global__ void __launch_bounds__(128, 1) score_tc_kernel(ScoreTcArgs a) {
                 tc_commit(bar_mma(s));
                 pending |= 8u << s;
                 ++issued_mma[s];
+                // the stage of tile n - 1 is free once its MMAs complete: refill it
+                // with tile n + 1 while tile n multiplies
+                if (n >= 1 && n + 1 < ntiles) {
+                    const int s1 = (int)((n + 1) & 1);
+                    if (mbar_wait(bar_mma(s1), (uint32_t)(((n - 1) >> 1) & 1))) {
+                        pending &= ~(8u << s1);
+                        fill(n + 1, s1);
+                    } else {
+                        ok = false;
+                    }
+                }
             }
         }
         // scores of tile n - 1 while tile n multiplies
@@ -374,14 +394,6 @@ __global__ void __launch_bounds__(128, 1) score_tc_kernel(ScoreTcArgs a) {
         if (s_fail) {
             ok = false;
             break;
-        }
-        // refill the stage of tile n - 1 (its MMAs finished: their commit was waited on)
-        if (tid == 0 && n >= 1 && n + 1 < ntiles) {
-            const int s1 = (int)((n + 1) & 1);
-            mbar_expect_tx(bar_full(s1), TC_BTILE);
-            bulk_g2s(smem_u32(sB + s1 * TC_BTILE), btree + (n + 1) * TC_BTILE, TC_BTILE, bar_full(s1));
-            pending |= 2u << s1;
-            ++issued_full[s1];
         }
     }
     if (ok && ntiles >= 1) epilogue(ntiles - 1);

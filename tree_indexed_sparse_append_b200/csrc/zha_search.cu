@@ -847,8 +847,10 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
         {
             Probe pr(t, ZHA_K_SELECT, st);
             if (t->n_nodes[l] > 8192) {
+                // few walks: the widest frontier sets the time, give it 1,024 threads;
+                // many walks (prefill): 512 threads keep two CTAs per SM
                 se.smem_keys = std::min<long long>(t->n_nodes[l], 16384);
-                e = launch_select<1024>(se, W, st);
+                e = W <= 2LL * num_sms() ? launch_select<1024>(se, W, st) : launch_select<512>(se, W, st);
             } else {
                 se.smem_keys = t->n_nodes[l];
                 e = launch_select<256>(se, W, st);
