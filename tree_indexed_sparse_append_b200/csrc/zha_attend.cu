@@ -119,6 +119,7 @@ __device__ __forceinline__ void block_scan2(long long &a, long long &b, long lon
 }
 
 __global__ void __launch_bounds__(1024) attend_plan_kernel(PlanArgs a) {
+    chain_start();
     __shared__ long long sh[64];
     // 1. the call's total key count sets the item length
     long long keys = 0;
@@ -169,6 +170,7 @@ __global__ void __launch_bounds__(1024) attend_plan_kernel(PlanArgs a) {
         a.item_off[a.W] = (int)icarry;
         a.group_off[a.W] = (int)gcarry;
     }
+    chain_done();
 }
 
 struct ItemArgs {
@@ -355,6 +357,7 @@ __device__ __forceinline__ int find_walk(const int *s_io, int W, long long item)
 
 template <typename T, int D, bool LOCAL>
 __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
+    chain_start();
     constexpr int EPL = Row<T>::EPL;
     constexpr int LPR0 = D / EPL;
     constexpr int LPR = LPR0 < 32 ? LPR0 : 32;  // lanes per row
@@ -583,6 +586,7 @@ __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
         merge_rows<D>(a.gpartial + g_first * PS, ngroups, lane, gm, gsum, o);
         write_out<D>(a, walk, lane, gm, gsum, o);
     }
+    chain_done();
 }
 
 template <typename T, int D, bool LOCAL>
@@ -600,8 +604,7 @@ cudaError_t launch_items(const zha_tree *t, const ItemArgs &ia, long long max_it
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     Probe pr(t, ZHA_K_ATTEND_PARTIAL, st);
-    attend_items_kernel<T, D, LOCAL><<<(unsigned)blocks, 256, smem, st>>>(ia);
-    return cudaGetLastError();
+    return launch_chained(attend_items_kernel<T, D, LOCAL>, dim3((unsigned)blocks), dim3(256), smem, st, ia);
 }
 
 template <typename T, int D>
@@ -611,6 +614,23 @@ cudaError_t launch_items_any(const zha_tree *t, const ItemArgs &ia, long long ma
 }
 
 }  // namespace
+
+namespace {
+__global__ void clear_kernel(int *p, long long n) {
+    chain_start();
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        p[i] = 0;
+    chain_done();
+}
+}  // namespace
+
+cudaError_t launch_clear(const zha_tree *t, int *p, long long n, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    long long blocks = (n + 255) / 256;
+    if (blocks > 4LL * num_sms()) blocks = 4LL * num_sms();
+    Probe pr(t, ZHA_K_ATTEND_PLAN, st);
+    return launch_chained(clear_kernel, dim3((unsigned)blocks), dim3(256), 0, st, p, n);
+}
 
 AttendLayout attend_layout(long long W, int D) {
     AttendLayout L{};
@@ -673,14 +693,12 @@ cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zh
     if (W <= LOCAL_MAX_W) {
         // the item kernel plans for itself; only the completion counters (walk
         // and group tickets, adjacent in the scratch) must start at zero
-        const size_t bytes = reinterpret_cast<const char *>(s.group_done + s.max_groups) -
-                             reinterpret_cast<const char *>(s.walk_done);
-        cudaError_t e = cudaMemsetAsync(s.walk_done, 0, bytes, st);
+        const long long words = reinterpret_cast<const int *>(s.group_done + s.max_groups) - s.walk_done;
+        cudaError_t e = launch_clear(t, s.walk_done, words, st);
         if (e != cudaSuccess) return e;
     } else {
         Probe pr(t, ZHA_K_ATTEND_PLAN, st);
-        attend_plan_kernel<<<1, 1024, 0, st>>>(pl);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_chained(attend_plan_kernel, dim3(1), dim3(1024), 0, st, pl);
         if (e != cudaSuccess) return e;
     }
 

@@ -37,6 +37,7 @@ struct BuildArgs {
 
 template <typename CT, int D>
 __global__ void __launch_bounds__(512) build_nodes_kernel(BuildArgs a) {
+    chain_start();
     constexpr int EPL = D / 32;
     extern __shared__ float smem[];
     const int lane = threadIdx.x & 31;
@@ -111,6 +112,7 @@ __global__ void __launch_bounds__(512) build_nodes_kernel(BuildArgs a) {
         if (lane == 0) node[a.R * D + r] = lse - a.beta * dq;
         __syncwarp();
     }
+    chain_done();
 }
 
 template <typename CT, int D>
@@ -129,18 +131,19 @@ cudaError_t launch_build_typed(const zha_tree *t, const BuildArgs &a, cudaStream
     if (blocks > cap) blocks = cap;
     if (blocks < 1) return cudaSuccess;
     Probe pr(t, ZHA_K_BUILD, st);
-    build_nodes_kernel<CT, D><<<(unsigned)blocks, threads, smem, st>>>(a);
-    return cudaGetLastError();
+    return launch_chained(build_nodes_kernel<CT, D>, dim3((unsigned)blocks), dim3(threads), smem, st, a);
 }
 
 template <typename T, int D>
 __global__ void append_kv_kernel(T *K, T *V, const T *k_new, const T *v_new, long long cap,
                                  long long n) {
+    chain_start();
     const int t = blockIdx.x;
     for (int e = threadIdx.x; e < D; e += blockDim.x) {
         K[((long long)t * cap + n) * D + e] = k_new[(long long)t * D + e];
         V[((long long)t * cap + n) * D + e] = v_new[(long long)t * D + e];
     }
+    chain_done();
 }
 
 }  // namespace
@@ -191,9 +194,10 @@ cudaError_t launch_append_kv(const zha_tree *t, const void *k_new, const void *v
     const zha_config &c = t->cfg;
     const int threads = c.d < 256 ? c.d : 256;
     Probe pr(t, ZHA_K_APPEND, st);
-#define ZHA_APPEND(TY, DD)                                                                         \
-    append_kv_kernel<TY, DD><<<t->T, threads, 0, st>>>((TY *)t->K, (TY *)t->V, (const TY *)k_new,  \
-                                                       (const TY *)v_new, c.capacity, t->n)
+    cudaError_t e = cudaSuccess;
+#define ZHA_APPEND(TY, DD)                                                                              \
+    e = launch_chained(append_kv_kernel<TY, DD>, dim3(t->T), dim3(threads), 0, st, (TY *)t->K, (TY *)t->V, \
+                       (const TY *)k_new, (const TY *)v_new, c.capacity, t->n)
     if (c.kv_dtype == ZHA_BF16) {
         if (c.d == 64) ZHA_APPEND(__nv_bfloat16, 64);
         else if (c.d == 128) ZHA_APPEND(__nv_bfloat16, 128);
@@ -204,7 +208,7 @@ cudaError_t launch_append_kv(const zha_tree *t, const void *k_new, const void *v
         else ZHA_APPEND(float, 256);
     }
 #undef ZHA_APPEND
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace zha

@@ -19,6 +19,15 @@ __device__ __forceinline__ void report(int *status, int code) {
     if (status) atomicCAS(status, DEV_OK, code);
 }
 
+// Kernels of one call chain (append, search, attend) are launched with
+// programmatic stream serialization (launch_chained): each first waits until the
+// grids before it have completed and their writes are visible (chain_start), so
+// nothing is read early and results are the same as with plain stream order;
+// each CTA lets the next grid be scheduled when its own work is done
+// (chain_done), so the next launch's latency overlaps this grid's tail.
+__device__ __forceinline__ void chain_start() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void chain_done() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------
 // Loads. Node data is streamed once per launch: keep it out of L1.
 __device__ __forceinline__ float4 ld_stream4(const float *p) {
@@ -261,6 +270,27 @@ cudaError_t launch_dense_scan(const zha_tree *t, const void *Q, zha_dtype q_dtyp
                               uint32_t *gkey, cudaStream_t st);
 
 int num_sms();
+
+// Launches kernel<<<grid, block, smem, st>>>(args...) with programmatic stream
+// serialization allowed (the kernel must begin with chain_start()).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                  Args... args) {
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Sets n ints to zero (a chained launch, where a memset would break the chain).
+cudaError_t launch_clear(const zha_tree *t, int *p, long long n, cudaStream_t st);
 
 // Every kernel launch is bracketed by probe_begin / probe_end: they count the
 // launch and, when the tree is being profiled, record a CUDA event pair.

@@ -89,9 +89,9 @@ extern "C" int zha_attend_noalloc(zha_tree *t, const void *Q, zha_dtype q_dtype,
 
     zha::Scratch s{};
     zha::attend_carve(layout, base, &s);
-    // The plan kernel writes every offset, item owner and item length the item
-    // kernel reads and zeroes the completion counters, so what an earlier call
-    // left in the array needs no clearing here.
+    // The attention clears its completion counters itself (a clear kernel, or the
+    // plan kernel for large calls) and computes every offset and item length it
+    // reads, so what an earlier call left in the array needs no clearing here.
 
     // The profiler's CUDA events are created on demand; keep it out of this call.
     zha_profiler *prof = t->prof;

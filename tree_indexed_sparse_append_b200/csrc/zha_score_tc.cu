@@ -93,7 +93,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
 
 __device__ __forceinline__ unsigned long long global_ns() {
     unsigned long long t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
 
