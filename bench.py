@@ -341,7 +341,7 @@ def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes
             tree.profile(False)
             kbytes = B * H * tree.n_keys * d * inp.K.element_size()
             r = results[mname]
-            search_ms = sum(r["kernel_ms_per_step"][k2] for k2 in ("search_init", "score", "select", "union"))
+            search_ms = sum(r["kernel_ms_per_step"][k2] for k2 in ("search_init", "score", "select", "score_tc"))
             dense[mname] = {"ms": ms, "key_read_gbs": kbytes / (ms / 1e3) / 1e9, "kernel_ms": dk,
                             "keys_selected_mean": float(dcnt.float().mean().item()),
                             "tree_search_ms": search_ms, "dense_over_tree_search": ms / search_ms}
@@ -447,11 +447,37 @@ def run_prefill(args, dev):
     tree.sync_status()
     walk_nodes = sum(info["walk_nodes"][1:info["start_level"] + 1])
     flops = 2.0 * w.R * w.d * walk_nodes
+    # levels scored on the tensor cores (trees of >= 1,024 bf16 walks, levels of
+    # <= 8,192 nodes, d = 128): every (walk, node, reference) of the level, each fp32
+    # key taken as three bf16 parts
+    G = Wk // (w.batch * w.n_kv_heads)
+    rp = 1
+    while rp < w.R:
+        rp *= 2
+    sizes = tree.level_sizes()
+    tc_ops = sum(2.0 * Wk * n * rp * w.d * 3 for l, n in enumerate(sizes[1:], start=1)
+                 if l <= info["start_level"] and 0 < n <= 8192 and G >= 1024 and w.d == 128
+                 and inp.Q.dtype == torch.bfloat16)
+    tc_ms = kt.get("score_tc")
+    bf16_peak = None
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16_peak = float(json.load(f)["bf16_tflops"])
+    except Exception:
+        pass
+    tensor = None
+    if tc_ms and tc_ops:
+        ach = tc_ops / (tc_ms / 1e3) / 1e12
+        tensor = {"bound": "tensor", "kernel": "score_tc", "achieved": ach, "peak": bf16_peak, "unit": "TFLOP/s",
+                  "frac": ach / bf16_peak if bf16_peak else None, "peak_source": "measured (burst)",
+                  "ops_per_step": tc_ops, "ms_per_step": tc_ms}
     res = {"workload": f"prefill: {w.queries_per_head:,} queries x 16 q-heads against the 4 KV-head trees of one "
                        "262,144-key sequence, d=128, bf16, C=8, depth 6, R=8, top-p 0.9",
            "walks": Wk, "ms": ms, "value": Wk / (ms / 1e3), "unit": UNIT, "kernel_ms": kt,
-           "score_tflops": flops / (kt["score"] / 1e3) / 1e12 if kt.get("score") else None,
-           "scored_walk_nodes": walk_nodes, "union_nodes": sum(info["union_nodes"][1:info["start_level"] + 1])}
+           "score_tflops": (flops / ((kt.get("score", 0) + kt.get("score_tc", 0)) / 1e3) / 1e12
+                            if kt.get("score") or kt.get("score_tc") else None),
+           "scored_walk_nodes": walk_nodes, "union_nodes": sum(info["union_nodes"][1:info["start_level"] + 1]),
+           "tensor_roofline": tensor}
     tree.close()
     del inp, sel, cnt, out, lse
     torch.cuda.empty_cache()

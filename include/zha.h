@@ -230,7 +230,7 @@ typedef enum {
     ZHA_K_ATTEND_PLAN = 5,    /* split of each walk's keys into work items */
     ZHA_K_ATTEND_PARTIAL = 6, /* gathered attention over the chosen keys */
     ZHA_K_ATTEND_COMBINE = 7, /* log-sum-exp merge of partial results (when a separate launch) */
-    ZHA_K_UNION = 8,          /* per-tree list of the union of the frontiers, one per level */
+    ZHA_K_SCORE_TC = 8,       /* tensor-core scoring of whole levels (prefill), with its tile preparation */
     ZHA_K_KINDS = 9
 } zha_kernel_kind;
 

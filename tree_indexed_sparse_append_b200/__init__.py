@@ -30,7 +30,7 @@ SYMBOLS = ("zha_build", "zha_append", "zha_search", "zha_attend", "zha_reserve",
            "zha_profile", "zha_profile_read", "zha_kernel_launches", "zha_last_search_info",
            "zha_dense_scan", "zha_attend_noalloc")
 KERNEL_KINDS = ("build", "append", "search_init", "score", "select", "attend_plan", "attend_partial",
-                "attend_combine", "union")
+                "attend_combine", "score_tc")
 
 
 class ZhaError(RuntimeError):

@@ -21,15 +21,16 @@
 //                    in the tensor cores' K-major core-matrix order (8 rows x 16 B
 //                    blocks), then the 128 biases (-inf for padding).
 //   tc_prep_queries  the tree's queries -> A tiles of 128 walks, same order.
-//   score_tc_kernel  one CTA per A tile: the A tile stays in shared memory, the B
-//                    tiles stream through a two-stage ring filled by bulk copies
-//                    (cp.async.bulk, no multicast; a stage is refilled as soon as
-//                    the MMAs reading it complete, the biases go to a ring of
-//                    their own), one thread issues the tcgen05.mma (M = N = 128,
-//                    K = 16, bf16 -> fp32 in TMEM) into two accumulators used in
-//                    turn, and four warps read a finished accumulator back
-//                    (tcgen05.ld), take the max over references and store the
-//                    scores.
+//   score_tc_kernel  one CTA per two A tiles (256 walks): both stay in shared
+//                    memory while the B tiles stream through a ring of four
+//                    32 KB part slots filled by bulk copies (cp.async.bulk, no
+//                    multicast), each slot refilled as soon as the MMAs reading it
+//                    complete. A producer warp issues the copies and the
+//                    tcgen05.mma (M = N = 128, K = 16, bf16 -> fp32 in TMEM), each
+//                    B part feeding both A tiles, into accumulators used in turn
+//                    (2 tiles x 2 buffers = all 512 TMEM columns); eight epilogue
+//                    warps read a finished accumulator back (tcgen05.ld), free it,
+//                    take the max over references and store the scores.
 // Every wait is bounded: on timeout the kernel records DEV_TIMEOUT, waits (also
 // bounded) for its own copies and MMAs, frees its TMEM and returns.
 #include <cstdint>
@@ -45,11 +46,11 @@ constexpr int TC_K = 128;                            // head dimension
 constexpr int TC_PART = TC_N * TC_K * 2;             // bytes of one bf16 part of a B tile
 constexpr int TC_BTILE = 3 * TC_PART + TC_N * 4;     // hi, mid, lo, biases
 constexpr int TC_ATILE = TC_M * TC_K * 2;
-constexpr int TC_STAGES = 2;
-constexpr int TC_BIAS_SLOTS = 4;                     // a tile's biases outlive its B stage
-constexpr int TC_STAGE = 3 * TC_PART;                // shared memory of one B stage (the three parts)
-constexpr int TC_SMEM = TC_ATILE + TC_STAGES * TC_STAGE + TC_BIAS_SLOTS * TC_N * 4 + 128;  // + barriers, TMEM address
-constexpr int TC_TMEM_COLS = 2 * TC_N;               // two fp32 accumulators of 128 columns
+constexpr int TC_MT = 2;                             // A tiles (of 128 walks) per CTA
+constexpr int TC_SLOTS = 4;                          // B part slots in shared memory
+constexpr int TC_SMEM = TC_MT * TC_ATILE + TC_SLOTS * TC_PART + 128;  // + barriers, TMEM address, flag
+constexpr int TC_TMEM_COLS = 512;                    // TC_MT x 2 fp32 accumulators of 128 columns
+constexpr int TC_THREADS = 9 * 32;                   // 8 epilogue warps + 1 producer warp
 constexpr unsigned long long TC_WAIT_NS = 1000000000ull;  // a wait gives up after 1 s
 
 // byte offset of element (row, k) in a 128-row K-major tile without swizzle:
@@ -230,7 +231,7 @@ __global__ void tc_prep_queries_kernel(PrepQArgs a, long long total) {
 
 struct ScoreTcArgs {
     const unsigned char *atiles, *btiles;
-    long long mtiles, ntiles, n_level;
+    long long mtiles, ntiles, n_level;  // mtiles: A tiles per tree, a multiple of TC_MT
     int G;
     float beta;
     float *S;
@@ -238,32 +239,47 @@ struct ScoreTcArgs {
     int *status;
 };
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 // RP: columns per node (R rounded up to a power of two; padded references have
 // zero keys and bias -inf)
 template <int RP>
-__global__ void __launch_bounds__(128, 1) score_tc_kernel(ScoreTcArgs a) {
+__global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(ScoreTcArgs a) {
     constexpr int NPT = TC_N / RP;  // nodes per B tile
     extern __shared__ __align__(16) unsigned char smem[];  // no static shared memory: all of it is here
-    unsigned char *sA = smem;
-    unsigned char *sB = smem + TC_ATILE;
-    float *sBias = reinterpret_cast<float *>(smem + TC_ATILE + TC_STAGES * TC_STAGE);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TC_ATILE + TC_STAGES * TC_STAGE + TC_BIAS_SLOTS * TC_N * 4);
-    // bars[0..1]: B stage s filled (bulk copies); bars[2..3]: accumulator s written
-    // (MMA commit); bars[4]: A tile filled
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
-    int &s_fail = *reinterpret_cast<int *>(bars + 7);
+    unsigned char *sA = smem;                              // TC_MT A tiles
+    unsigned char *sB = smem + TC_MT * TC_ATILE;           // TC_SLOTS B part slots
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TC_MT * TC_ATILE + TC_SLOTS * TC_PART);
+    // bars 0-3: slot filled; 4-7: slot's MMAs done; 8-9: accumulator buffer written
+    // (MMA commit); 10-11: accumulator buffer read back (8 warps); 12: A tiles
+    // filled; 13: all MMAs done (cleanup)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
+    volatile int *fail = reinterpret_cast<volatile int *>(bars + 15);
 
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const long long mt = blockIdx.x, t = blockIdx.y;
-    const long long ntiles = a.ntiles;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long ct = blockIdx.x, t = blockIdx.y;
+    const long long ntiles = a.ntiles, nparts = 3 * ntiles;
     const unsigned char *btree = a.btiles + t * ntiles * TC_BTILE;
-    const uint32_t barA = smem_u32(bars + 4);
-    auto bar_full = [&](int s) { return smem_u32(bars + s); };
-    auto bar_mma = [&](int s) { return smem_u32(bars + 2 + s); };
+    auto full = [&](int s) { return smem_u32(bars + s); };
+    auto empty = [&](int s) { return smem_u32(bars + 4 + s); };
+    auto accf = [&](int b) { return smem_u32(bars + 8 + b); };
+    auto accfree = [&](int b) { return smem_u32(bars + 10 + b); };
+    const uint32_t barA = smem_u32(bars + 12), barEnd = smem_u32(bars + 13);
 
     if (tid == 0) {
-        s_fail = 0;
-        for (int i = 0; i < 5; ++i) mbar_init(smem_u32(bars + i), 1);
+        *fail = 0;
+        for (int i = 0; i < TC_SLOTS; ++i) {
+            mbar_init(full(i), 1);
+            mbar_init(empty(i), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(accf(b), 1);
+            mbar_init(accfree(b), 8);
+        }
+        mbar_init(barA, 1);
+        mbar_init(barEnd, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -277,137 +293,136 @@ __global__ void __launch_bounds__(128, 1) score_tc_kernel(ScoreTcArgs a) {
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // thread 0 issues every copy and MMA and remembers which are still in flight:
-    // bit 0: A copy; bits 1..2: B stage copies; bits 3..4: MMA groups
-    unsigned pending = 0;
-    long long issued_full[TC_STAGES] = {0, 0}, issued_mma[TC_STAGES] = {0, 0};  // uses so far, per barrier
-    // B tile n -> stage s: its three parts into the stage, its biases into slot n % 4
-    auto fill = [&](long long n, int s) {
-        const unsigned char *src = btree + n * TC_BTILE;
-        mbar_expect_tx(bar_full(s), TC_BTILE);
-        bulk_g2s(smem_u32(sB + s * TC_STAGE), src, TC_STAGE, bar_full(s));
-        bulk_g2s(smem_u32(sBias + (n & (TC_BIAS_SLOTS - 1)) * TC_N), src + TC_STAGE, TC_N * 4, bar_full(s));
-        pending |= 2u << s;
-        ++issued_full[s];
-    };
-    if (tid == 0) {
-        mbar_expect_tx(barA, TC_ATILE);
-        bulk_g2s(smem_u32(sA), a.atiles + (t * a.mtiles + mt) * TC_ATILE, TC_ATILE, barA);
-        pending |= 1u;
-        for (int s = 0; s < TC_STAGES && s < ntiles; ++s) fill(s, s);
-    }
-
-    const long long g = mt * TC_M + tid;  // this thread's walk within the tree (row of the tile)
-    const bool row_ok = g < a.G;
-    float *Srow = a.S + (t * a.G + (row_ok ? g : 0)) * a.Sstride;
-    const bool vec_ok = (a.Sstride & 3) == 0;
-    bool ok = true;
-
-    // reads accumulator (n & 1) of tile n and writes its scores
-    auto epilogue = [&](long long n) {
-        const int s = (int)(n & 1);
-        if (ok) {
-            if (mbar_wait(bar_mma(s), (uint32_t)((n >> 1) & 1))) {
-                if (tid == 0) pending &= ~(8u << s);
-            } else {
-                ok = false;
-            }
-        }
-        tc_fence_after();
-        const float *bias = sBias + (n & (TC_BIAS_SLOTS - 1)) * TC_N;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(s * TC_N);
-        float sc[TC_N];
-#pragma unroll
-        for (int c0 = 0; c0 < TC_N; c0 += 16) {
-            float v[16];
-            tc_ld16(lane_base + c0, v);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) sc[c0 + i] = v[i];
-        }
-        tc_wait_ld();
-        // node q's score goes to sc[q] (q <= q * RP, so no later read is overwritten)
-#pragma unroll
-        for (int q = 0; q < NPT; ++q) {
-            float m = -INFINITY;
-#pragma unroll
-            for (int r = 0; r < RP; ++r) m = fmaxf(m, fmaf(a.beta, sc[q * RP + r], bias[q * RP + r]));
-            sc[q] = m;
-        }
-        if (ok && row_ok) {
-            const long long j0 = n * NPT;
-#pragma unroll
-            for (int q = 0; q < NPT; q += 4) {
-                if (NPT >= 4 && vec_ok && j0 + q + 3 < a.n_level) {
-                    *reinterpret_cast<float4 *>(Srow + j0 + q) = make_float4(sc[q], sc[q + 1], sc[q + 2], sc[q + 3]);
-                } else {
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        if (q + u < NPT && j0 + q + u < a.n_level) Srow[j0 + q + u] = sc[q + u];
+    if (warp == 8) {
+        // producer: one thread issues every copy and MMA
+        if (lane == 0) {
+            bool ok = true;
+            long long fills[TC_SLOTS] = {0, 0, 0, 0}, waited[TC_SLOTS] = {0, 0, 0, 0};
+            bool a_waited = false, any_mma = false;
+            auto fill = [&](long long j) {  // B part j -> slot j % 4
+                const int s = (int)(j & (TC_SLOTS - 1));
+                mbar_expect_tx(full(s), TC_PART);
+                bulk_g2s(smem_u32(sB + s * TC_PART), btree + (j / 3) * TC_BTILE + (j % 3) * TC_PART, TC_PART, full(s));
+                ++fills[s];
+            };
+            mbar_expect_tx(barA, TC_MT * TC_ATILE);
+            bulk_g2s(smem_u32(sA), a.atiles + (t * a.mtiles + TC_MT * ct) * TC_ATILE, TC_MT * TC_ATILE, barA);
+            for (long long j = 0; j < TC_SLOTS && j < nparts; ++j) fill(j);
+            if (mbar_wait(barA, 0)) a_waited = true;
+            else ok = false;
+            for (long long n = 0; ok && n < ntiles; ++n) {
+                const int b = (int)(n & 1);
+                // accumulator buffer b is free once the epilogue of tile n - 2 read it
+                if (n >= 2 && !mbar_wait(accfree(b), (uint32_t)(((n - 2) >> 1) & 1))) {
+                    ok = false;
+                    break;
                 }
-            }
-        }
-        tc_fence_before();
-    };
-
-    if (tid == 0) {
-        if (mbar_wait(barA, 0)) pending &= ~1u;
-        else ok = false;
-    }
-    for (long long n = 0; n < ntiles; ++n) {
-        const int s = (int)(n & 1);
-        // MMA for tile n into accumulator s (free: the epilogue of its previous tile
-        // ended before the last block barrier)
-        if (tid == 0 && ok) {
-            if (!mbar_wait(bar_full(s), (uint32_t)((n >> 1) & 1))) {
-                ok = false;
-            } else {
-                pending &= ~(2u << s);
                 tc_fence_after();
-                const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB + s * TC_STAGE);
-                const uint32_t d = tmem + (uint32_t)(s * TC_N);
-#pragma unroll
-                for (int part = 0; part < 3; ++part)
-#pragma unroll
-                    for (int ks = 0; ks < TC_K / 16; ++ks)
-                        tc_mma(d, smem_desc(a0 + ks * 256), smem_desc(b0 + part * TC_PART + ks * 256),
-                               (part | ks) ? 1u : 0u);
-                tc_commit(bar_mma(s));
-                pending |= 8u << s;
-                ++issued_mma[s];
-                // the stage of tile n - 1 is free once its MMAs complete: refill it
-                // with tile n + 1 while tile n multiplies
-                if (n >= 1 && n + 1 < ntiles) {
-                    const int s1 = (int)((n + 1) & 1);
-                    if (mbar_wait(bar_mma(s1), (uint32_t)(((n - 1) >> 1) & 1))) {
-                        pending &= ~(8u << s1);
-                        fill(n + 1, s1);
-                    } else {
+                for (int p = 0; p < 3; ++p) {
+                    const long long j = 3 * n + p;
+                    const int s = (int)(j & (TC_SLOTS - 1));
+                    if (!mbar_wait(full(s), (uint32_t)((j >> 2) & 1))) {
                         ok = false;
+                        break;
+                    }
+                    ++waited[s];
+                    tc_fence_after();
+                    const uint32_t b0 = smem_u32(sB + s * TC_PART);
+#pragma unroll
+                    for (int m = 0; m < TC_MT; ++m) {
+                        const uint32_t a0 = smem_u32(sA + m * TC_ATILE);
+                        const uint32_t d = tmem + (uint32_t)((2 * m + b) * TC_N);
+#pragma unroll
+                        for (int ks = 0; ks < TC_K / 16; ++ks)
+                            tc_mma(d, smem_desc(a0 + ks * 256), smem_desc(b0 + ks * 256), (p | ks) ? 1u : 0u);
+                    }
+                    any_mma = true;
+                    tc_commit(empty(s));
+                    if (p == 2) tc_commit(accf(b));
+                    // the slot of part j - 1 is free once its MMAs complete (part j's
+                    // are queued behind them): refill it with part j + 3
+                    if (j >= 1 && j + 3 < nparts) {
+                        const int s1 = (int)((j - 1) & (TC_SLOTS - 1));
+                        if (!mbar_wait(empty(s1), (uint32_t)(((j - 1) >> 2) & 1))) {
+                            ok = false;
+                            break;
+                        }
+                        fill(j + 3);
                     }
                 }
             }
+            if (!ok) {
+                *fail = 1;
+                report(a.status, DEV_TIMEOUT);
+                // let the copies and MMAs in flight finish (bounded waits)
+                if (!a_waited) (void)mbar_wait(barA, 0);
+                for (int s = 0; s < TC_SLOTS; ++s)
+                    if (fills[s] > waited[s]) (void)mbar_wait(full(s), (uint32_t)((fills[s] - 1) & 1));
+                if (any_mma) {
+                    tc_commit(barEnd);
+                    (void)mbar_wait(barEnd, 0);
+                }
+            }
         }
-        // scores of tile n - 1 while tile n multiplies
-        if (n >= 1) epilogue(n - 1);
-        if (!ok) s_fail = 1;
-        __syncthreads();
-        if (s_fail) {
-            ok = false;
-            break;
-        }
-    }
-    if (ok && ntiles >= 1) epilogue(ntiles - 1);
-    if (!ok) s_fail = 1;
-    __syncthreads();
-    if (s_fail) {
-        // let the copies and MMAs still in flight finish before the memory they
-        // write is released (each wait bounded as well)
-        if (tid == 0) {
-            report(a.status, DEV_TIMEOUT);
-            if (pending & 1u) (void)mbar_wait(barA, 0);
-            for (int s = 0; s < TC_STAGES; ++s) {
-                if (pending & (2u << s)) (void)mbar_wait(bar_full(s), (uint32_t)((issued_full[s] - 1) & 1));
-                if (pending & (8u << s)) (void)mbar_wait(bar_mma(s), (uint32_t)((issued_mma[s] - 1) & 1));
+    } else {
+        // epilogue: warps 0-3 read A tile 0's accumulators, warps 4-7 A tile 1's;
+        // a warp reads TMEM lanes 32 * (warp % 4) .. + 31 (one walk per lane)
+        const int m = warp >> 2, wq = warp & 3;
+        const long long g = (TC_MT * ct + m) * TC_M + wq * 32 + lane;
+        const bool row_ok = g < a.G;
+        float *Srow = a.S + (t * a.G + (row_ok ? g : 0)) * a.Sstride;
+        const bool vec_ok = (a.Sstride & 3) == 0;
+        for (long long n = 0; n < ntiles; ++n) {
+            const int b = (int)(n & 1);
+            if (!mbar_wait(accf(b), (uint32_t)((n >> 1) & 1)) || *fail) break;
+            tc_fence_after();
+            const uint32_t base = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)((2 * m + b) * TC_N);
+            float sc[TC_N];
+#pragma unroll
+            for (int c0 = 0; c0 < TC_N; c0 += 16) {
+                float v[16];
+                tc_ld16(base + c0, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sc[c0 + i] = v[i];
+            }
+            tc_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(accfree(b));
+            const float4 *bias4 = reinterpret_cast<const float4 *>(btree + n * TC_BTILE + 3 * TC_PART);
+            // node q's score goes to sc[q] (q <= q * RP, so no later read is overwritten)
+#pragma unroll
+            for (int q = 0; q < NPT; ++q) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int r4 = 0; r4 < RP; r4 += 4) {
+                    const int c = q * RP + r4;
+                    float bb[4];
+                    if (RP >= 4) {
+                        const float4 v = __ldg(bias4 + c / 4);
+                        bb[0] = v.x, bb[1] = v.y, bb[2] = v.z, bb[3] = v.w;
+                    } else {
+                        const float *bias = reinterpret_cast<const float *>(bias4);
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) bb[r] = r < RP ? __ldg(bias + c + r) : 0.f;
+                    }
+#pragma unroll
+                    for (int r = 0; r < 4 && r < RP; ++r) mx = fmaxf(mx, fmaf(a.beta, sc[c + r], bb[r]));
+                }
+                sc[q] = mx;
+            }
+            if (row_ok) {
+                const long long j0 = n * NPT;
+#pragma unroll
+                for (int q = 0; q < NPT; q += 4) {
+                    if (NPT >= 4 && vec_ok && j0 + q + 3 < a.n_level) {
+                        *reinterpret_cast<float4 *>(Srow + j0 + q) = make_float4(sc[q], sc[q + 1], sc[q + 2], sc[q + 3]);
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            if (q + u < NPT && j0 + q + u < a.n_level) Srow[j0 + q + u] = sc[q + u];
+                    }
+                }
             }
         }
     }
@@ -424,7 +439,7 @@ __global__ void __launch_bounds__(128, 1) score_tc_kernel(ScoreTcArgs a) {
 size_t tc_scratch_bytes(int T, long long G, long long max_level_nodes, int R) {
     int RP = 1;
     while (RP < R) RP <<= 1;
-    const long long mtiles = (G + TC_M - 1) / TC_M;
+    const long long mtiles = (G + TC_M * TC_MT - 1) / (TC_M * TC_MT) * TC_MT;
     const long long ntiles = (max_level_nodes * RP + TC_N - 1) / TC_N;
     return (size_t)T * mtiles * TC_ATILE + (size_t)T * ntiles * TC_BTILE;
 }
@@ -444,8 +459,8 @@ cudaError_t launch_score_tc_rp(const zha_tree *t, const ScoreTcArgs &sa, cudaStr
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    Probe pr(t, ZHA_K_SCORE, st);
-    score_tc_kernel<RP><<<dim3((unsigned)sa.mtiles, (unsigned)t->T), 128, TC_SMEM, st>>>(sa);
+    Probe pr(t, ZHA_K_SCORE_TC, st);
+    score_tc_kernel<RP><<<dim3((unsigned)(sa.mtiles / TC_MT), (unsigned)t->T), TC_THREADS, TC_SMEM, st>>>(sa);
     return cudaGetLastError();
 }
 }  // namespace
@@ -454,10 +469,10 @@ cudaError_t launch_score_tc_queries(const zha_tree *t, const void *Q, int G, uns
     PrepQArgs q{};
     q.Q = static_cast<const __nv_bfloat16 *>(Q);
     q.G = G;
-    q.mtiles = (G + TC_M - 1) / TC_M;
+    q.mtiles = (G + TC_M * TC_MT - 1) / (TC_M * TC_MT) * TC_MT;
     q.tiles = ws;
     const long long total = (long long)t->T * q.mtiles * TC_M * 16;
-    Probe pr(t, ZHA_K_SCORE, st);
+    Probe pr(t, ZHA_K_SCORE_TC, st);
     tc_prep_queries_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(q, total);
     return cudaGetLastError();
 }
@@ -467,7 +482,7 @@ cudaError_t launch_score_tc(const zha_tree *t, int level, int G, unsigned char *
     const zha_config &c = t->cfg;
     int RP = 1;
     while (RP < c.R) RP <<= 1;
-    const long long mtiles = (G + TC_M - 1) / TC_M;
+    const long long mtiles = (G + TC_M * TC_MT - 1) / (TC_M * TC_MT) * TC_MT;
     const long long n_level = t->n_nodes[level];
     const long long ntiles = (n_level * RP + TC_N - 1) / TC_N;
     unsigned char *atiles = ws;
@@ -485,7 +500,7 @@ cudaError_t launch_score_tc(const zha_tree *t, int level, int G, unsigned char *
     k.tiles = btiles;
     const long long total = (long long)t->T * ntiles * TC_N * 16;
     {
-        Probe pr(t, ZHA_K_SCORE, st);
+        Probe pr(t, ZHA_K_SCORE_TC, st);
         tc_prep_keys_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(k, total);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
