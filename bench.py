@@ -447,17 +447,24 @@ def run_prefill(args, dev):
     tree.sync_status()
     walk_nodes = sum(info["walk_nodes"][1:info["start_level"] + 1])
     flops = 2.0 * w.R * w.d * walk_nodes
-    # levels scored on the tensor cores (trees of >= 1,024 bf16 walks, levels of
-    # <= 8,192 nodes, d = 128): every (walk, node, reference) of the level, each fp32
-    # key taken as three bf16 parts
+    # levels scored on the tensor cores (trees of >= 1,024 bf16 walks, d = 128), each
+    # fp32 key taken as three bf16 parts: levels of <= 8,192 nodes as the dense
+    # contraction (every walk x node x reference), larger levels sparsely (counted
+    # as the frontier pairs they must score)
     G = Wk // (w.batch * w.n_kv_heads)
     rp = 1
     while rp < w.R:
         rp *= 2
     sizes = tree.level_sizes()
-    tc_ops = sum(2.0 * Wk * n * rp * w.d * 3 for l, n in enumerate(sizes[1:], start=1)
-                 if l <= info["start_level"] and 0 < n <= 8192 and G >= 1024 and w.d == 128
-                 and inp.Q.dtype == torch.bfloat16)
+    tc_ops = 0.0
+    if G >= 1024 and w.d == 128 and inp.Q.dtype == torch.bfloat16:
+        for l, n in enumerate(sizes[1:], start=1):
+            if l > info["start_level"] or n == 0:
+                continue
+            if n <= 8192:
+                tc_ops += 2.0 * Wk * n * rp * w.d * 3
+            elif w.R > 2:
+                tc_ops += 2.0 * info["walk_nodes"][l] * rp * w.d * 3
     tc_ms = kt.get("score_tc")
     bf16_peak = None
     try:

@@ -2,11 +2,15 @@
 the oracle, and agreement with the CUDA-core scorer on the same query values.
 
 The workload: one sequence, 2 KV heads and 4 query heads (2:1), 550 queries per
-query head, so 1,100 walks per tree (not a multiple of the 128-walk tile); 16,427
-clustered keys (blocks of 64 around random centres) with C = 8 and depth 4, so
-level sizes 2,053 / 256 / 32 / 4 and a ragged tail of 3 keys; R = 6 reference
-queries (padded to 8 columns per node); d = 128, bf16 keys, values and queries.
-Every level the walk visits is scored on the tensor cores.
+query head, so 1,100 walks per tree (not a multiple of the 128-walk tile);
+clustered keys (blocks of 64 around random centres) with C = 8 and depth 4; R = 6
+reference queries (padded to 8 columns per node); d = 128, bf16 keys, values and
+queries. Two tree sizes:
+  * 16,427 keys: level sizes 2,053 / 256 / 32 / 4, tail of 3 keys; every level the
+    walk visits is scored densely (all walks x all nodes);
+  * 70,003 keys: level sizes 8,750 / 1,093 / 136 / 17, tail of 3 keys; level 1
+    (more than 8,192 nodes) is scored sparsely (per tile of 16 nodes, only the
+    walks whose frontier holds one of them), the others densely.
 """
 import numpy as np
 import pytest
@@ -17,7 +21,7 @@ from helpers import assert_attention_close, compare_selection, host64, near_tie
 
 pytestmark = pytest.mark.gpu
 
-N, C, DEPTH, D, R, H, HQ, NQ = 16427, 8, 4, 128, 6, 2, 4, 550
+C, DEPTH, D, R, H, HQ, NQ = 8, 4, 128, 6, 2, 4, 550
 BETA = 1 / np.sqrt(D)
 
 
@@ -27,7 +31,7 @@ def zha():
     return Z
 
 
-def inputs(seed=7):
+def inputs(N, seed=7):
     g = torch.Generator(device="cuda").manual_seed(seed)
     blocks = (N + 63) // 64
     centres = torch.randn(H, blocks, D, generator=g, device="cuda")
@@ -56,10 +60,11 @@ def sample_walks():
     return sorted(picks)
 
 
+@pytest.mark.parametrize("N", [16427, 70003])
 @pytest.mark.parametrize("mode,p,k", [(O.TOP_P, 0.9, 0), (O.TOP_K, 0, 8)])
-def test_tensor_core_search_matches_oracle(mode, p, k):
+def test_tensor_core_search_matches_oracle(mode, p, k, N):
     Z = zha()
-    K, V, refs, Q = inputs()
+    K, V, refs, Q = inputs(N)
     tree = Z.Tree(K, V, refs, N, C, DEPTH, BETA)
     max_sel = N // C
     sel, cnt, st = tree.search(Q, mode, p, k, max_sel=max_sel, with_stats=True)
@@ -84,6 +89,13 @@ def test_tensor_core_search_matches_oracle(mode, p, k):
         assert_attention_close(out[wi], lse[wi], o_out, o_lse, 3e-3, f"walk {wi}")
         checked += 1
     assert checked > 0.9 * len(sample_walks())
+
+    # every level went through a tensor-core path (dense, or sparse above 8,192 nodes)
+    tree.profile(True)
+    tree.search(Q, mode, p, k, max_sel=max_sel)
+    kinds = tree.profile_read()
+    tree.profile(False)
+    assert kinds["score"][0] == 0 and kinds["score_tc"][0] > 0, kinds
 
     # the same query values as fp32 take the CUDA-core scorer
     sel2, cnt2, _ = tree.search(Q.float(), mode, p, k, max_sel=max_sel)

@@ -166,13 +166,16 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     const size_t o_att = take(att.bytes);
     // tensor-core scoring tiles, for trees walked by many queries
     const long long Gw = W / t->T;
-    size_t tc_bytes = 0;
+    TcLayout tcl{};
     if (c.d == 128 && Gw >= TC_MIN_G) {
-        long long maxn = 0;
-        for (int l = 1; l <= c.depth; ++l) maxn = std::max(maxn, std::min(t->cap_nodes[l], TC_MAX_NODES));
-        if (maxn > 0) tc_bytes = tc_scratch_bytes(t->T, Gw, maxn, c.R);
+        long long maxn_b = 0, maxn_sparse = 0;
+        for (int l = 1; l <= c.depth; ++l) {
+            maxn_b = std::max(maxn_b, t->cap_nodes[l]);
+            if (t->cap_nodes[l] > TC_MAX_NODES) maxn_sparse = std::max(maxn_sparse, t->cap_nodes[l]);
+        }
+        if (maxn_b > 0) tcl = tc_layout(t->T, Gw, maxn_b, maxn_sparse, c.R);
     }
-    const size_t o_tc = take(tc_bytes);
+    const size_t o_tc = take(tcl.bytes);
     const size_t need = off;
 
     if (need > t->ws_bytes) {
@@ -203,7 +206,11 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     s->M_bytes = M_bytes;
     s->U_bytes = U_bytes;
     attend_carve(att, b + o_att, s);
-    s->tc = tc_bytes ? reinterpret_cast<unsigned char *>(b + o_tc) : nullptr;
+    s->tc = tcl.bytes ? reinterpret_cast<unsigned char *>(b + o_tc + tcl.a_off) : nullptr;
+    s->tc_b = tcl.bytes ? reinterpret_cast<unsigned char *>(b + o_tc + tcl.b_off) : nullptr;
+    s->tc_counts = tcl.bytes && tcl.lists_off > tcl.counts_off ? reinterpret_cast<int *>(b + o_tc + tcl.counts_off)
+                                                                : nullptr;
+    s->tc_lists = tcl.bytes && tcl.bytes > tcl.lists_off ? reinterpret_cast<int *>(b + o_tc + tcl.lists_off) : nullptr;
     s->Sstride = cap1;
     s->Lstride = cap2;
     return ZHA_OK;

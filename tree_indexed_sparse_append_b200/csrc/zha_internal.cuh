@@ -221,7 +221,9 @@ struct Scratch {
     int *group_done;           // [max_groups] attend items finished per group
     float *partial;            // [max_items][D + 4]
     float *gpartial;           // [max_groups][D + 4]
-    unsigned char *tc;         // tensor-core scoring tiles (NULL when the walks per tree are few)
+    unsigned char *tc;         // tensor-core scoring: A tiles (NULL when the walks per tree are few)
+    unsigned char *tc_b;       //   B tiles of the level being scored
+    int *tc_counts, *tc_lists; //   per B tile: how many walks, and which, have one of its nodes in their frontier
     long long Sstride, Lstride, max_items, max_groups;
 };
 
@@ -240,13 +242,25 @@ void attend_carve(const AttendLayout &L, void *base, Scratch *s);
 // Tensor-core scoring of a whole level (zha_score_tc.cu), used for trees of at
 // least TC_MIN_G walks, levels of at most TC_MAX_NODES nodes, d = 128 and bf16
 // queries; other calls score on the CUDA cores.
+// Larger levels are scored sparsely on the tensor cores: per tile of nodes, only
+// the walks whose frontier holds one of its nodes (zha_score_tc.cu).
 constexpr int TC_MIN_G = 1024;
 constexpr long long TC_MAX_NODES = 8192;
-size_t tc_scratch_bytes(int T, long long G, long long max_level_nodes, int R);
+struct TcLayout {
+    size_t a_off, b_off, counts_off, lists_off, bytes;
+};
+// scratch of tensor-core scoring for trees of G walks: A tiles, the B tiles of the
+// widest level (maxn_b nodes), membership lists for a sparse level of maxn_sparse
+// nodes (0: none)
+TcLayout tc_layout(int T, long long G, long long maxn_b, long long maxn_sparse, int R);
 bool tc_applicable(const zha_tree *t, int G, const void *Q, zha_dtype q_dtype, int level);
+bool tc_sparse_applicable(const zha_tree *t, int G, const void *Q, zha_dtype q_dtype, int level);
 cudaError_t launch_score_tc_queries(const zha_tree *t, const void *Q, int G, unsigned char *ws, cudaStream_t st);
-cudaError_t launch_score_tc(const zha_tree *t, int level, int G, unsigned char *ws, float *S, long long Sstride,
-                            cudaStream_t st);
+cudaError_t launch_score_tc(const zha_tree *t, int level, int G, unsigned char *atiles, unsigned char *btiles,
+                            float *S, long long Sstride, cudaStream_t st);
+cudaError_t launch_score_tc_sparse(const zha_tree *t, int level, int G, const void *Q, const unsigned *M,
+                                   long long words, unsigned char *btiles, int *counts, int *lists, float *S,
+                                   long long Sstride, cudaStream_t st);
 // Records an error message for zha_last_error (this host thread); returns code.
 int set_error(int code, const char *msg);
 

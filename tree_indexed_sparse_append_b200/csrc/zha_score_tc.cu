@@ -436,17 +436,288 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(ScoreTcArgs a) 
 
 }  // namespace
 
-size_t tc_scratch_bytes(int T, long long G, long long max_level_nodes, int R) {
+namespace {
+
+// level keys -> B tiles (ntiles per tree)
+cudaError_t launch_prep_keys(const zha_tree *t, int level, int RP, long long ntiles, unsigned char *btiles,
+                             cudaStream_t st) {
+    const zha_config &c = t->cfg;
+    PrepKeysArgs k{};
+    k.nodes = t->nodes[level];
+    k.node_tree = t->cap_nodes[level] * t->NF;
+    k.NF = t->NF;
+    k.R = c.R;
+    k.RP = RP;
+    k.D = c.d;
+    k.n_level = t->n_nodes[level];
+    k.ntiles = ntiles;
+    k.tiles = btiles;
+    const long long total = (long long)t->T * ntiles * TC_N * 16;
+    Probe pr(t, ZHA_K_SCORE_TC, st);
+    tc_prep_keys_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(k, total);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Sparse levels: per B tile (NPT consecutive nodes, which share one membership
+// word), the walks of the tree whose frontier holds one of its nodes, in
+// ascending order; then one CTA per B tile multiplies the tile by those walks'
+// queries, 128 at a time, gathered into shared memory.
+struct MembersArgs {
+    const unsigned *M;  // level membership bits [T][words][G]
+    long long words, ntiles;
+    int G, NPT;
+    int *counts, *lists;  // [T][ntiles], [T][ntiles][G]
+};
+
+__global__ void __launch_bounds__(256) tc_members_kernel(MembersArgs a) {
+    __shared__ int s_warp[8];
+    const long long nt = blockIdx.x, t = blockIdx.y;
+    const long long n0 = nt * a.NPT;
+    const unsigned mask = a.NPT >= 32 ? 0xffffffffu : (((1u << a.NPT) - 1u) << (int)(n0 & 31));
+    const unsigned *Mrow = a.M + ((long long)t * a.words + (n0 >> 5)) * a.G;
+    int *list = a.lists + (t * a.ntiles + nt) * a.G;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int base = 0;
+    for (int g0 = 0; g0 < a.G; g0 += 256) {
+        const int g = g0 + threadIdx.x;
+        const bool member = g < a.G && (Mrow[g] & mask) != 0u;
+        const unsigned bal = __ballot_sync(FULL, member);
+        if (lane == 0) s_warp[wid] = __popc(bal);
+        __syncthreads();
+        int before = 0, total = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int c = s_warp[i];
+            before += i < wid ? c : 0;
+            total += c;
+        }
+        if (member) list[base + before + __popc(bal & ((1u << lane) - 1u))] = g;
+        base += total;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) a.counts[t * a.ntiles + nt] = base;
+}
+
+struct SparseArgs {
+    const unsigned char *btiles;  // [T][ntiles][TC_BTILE]
+    const __nv_bfloat16 *Q;       // [T * G][128]
+    const int *counts, *lists;
+    long long ntiles, n_level;
+    int G;
+    float beta;
+    float *S;
+    long long Sstride;
+    int *status;
+};
+
+constexpr int TS_SMEM = 3 * TC_PART + TC_ATILE + TC_N * 4 + 64;  // B tile, gathered walks, biases, barriers
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+template <int RP>
+__global__ void __launch_bounds__(128, 1) score_tc_sparse_kernel(SparseArgs a) {
+    constexpr int NPT = TC_N / RP;
+    extern __shared__ __align__(16) unsigned char smem[];  // no static shared memory: all of it is here
+    unsigned char *sB = smem;                              // the tile's three key parts
+    unsigned char *sA = smem + 3 * TC_PART;                // 128 gathered queries
+    float *sBias = reinterpret_cast<float *>(smem + 3 * TC_PART + TC_ATILE);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 3 * TC_PART + TC_ATILE + TC_N * 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const long long nt = blockIdx.x, t = blockIdx.y;
+    const long long tn = t * a.ntiles + nt;
+    const int count = a.counts[tn];
+    if (count <= 0) return;  // the same for the whole CTA; nothing allocated yet
+    const int *list = a.lists + tn * a.G;
+    const uint32_t barB = smem_u32(bars), barM = smem_u32(bars + 1);
+
+    if (tid == 0) {
+        mbar_init(barB, 1);
+        mbar_init(barM, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TC_N)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (tid == 0) {
+        const unsigned char *src = a.btiles + tn * TC_BTILE;
+        mbar_expect_tx(barB, 3 * TC_PART + TC_N * 4);
+        bulk_g2s(smem_u32(sB), src, 3 * TC_PART, barB);
+        bulk_g2s(smem_u32(sBias), src + 3 * TC_PART, TC_N * 4, barB);
+    }
+    bool ok = mbar_wait(barB, 0);
+    bool b_done = ok, m_pending = false;
+    uint32_t phase = 0;
+    for (int c0 = 0; c0 < count; c0 += TC_M) {
+        if (!__syncthreads_and(ok)) {
+            ok = false;
+            break;
+        }
+        const int rows = min(TC_M, count - c0);
+        // gather: thread i brings walk list[c0 + i]'s query (zeros past the list)
+        const int g = tid < rows ? list[c0 + tid] : -1;
+        const __nv_bfloat16 *src = a.Q + ((long long)t * a.G + (g >= 0 ? g : 0)) * TC_K;
+        const uint32_t dst = smem_u32(sA);
+#pragma unroll
+        for (int kc = 0; kc < TC_K / 8; ++kc) cp_async16(dst + core_offset(tid, kc * 8), src + kc * 8, g >= 0 ? 16u : 0u);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic-proxy writes -> MMA reads
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+#pragma unroll
+            for (int part = 0; part < 3; ++part)
+#pragma unroll
+                for (int ks = 0; ks < TC_K / 16; ++ks)
+                    tc_mma(tmem, smem_desc(a0 + ks * 256), smem_desc(b0 + part * TC_PART + ks * 256),
+                           (part | ks) ? 1u : 0u);
+            tc_commit(barM);
+        }
+        // one thread waits for the MMAs and tells the others, so that every warp
+        // takes the same branch before the warp-collective TMEM loads
+        volatile int *s_ok = reinterpret_cast<volatile int *>(bars + 3);
+        if (tid == 0) *s_ok = mbar_wait(barM, phase) ? 1 : 0;
+        __syncthreads();
+        if (!*s_ok) {
+            ok = false;
+            m_pending = true;
+            break;
+        }
+        phase ^= 1u;
+        tc_fence_after();
+        float sc[TC_N];
+#pragma unroll
+        for (int cc = 0; cc < TC_N; cc += 16) {
+            float v[16];
+            tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)cc, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sc[cc + i] = v[i];
+        }
+        tc_wait_ld();
+        tc_fence_before();
+#pragma unroll
+        for (int q = 0; q < NPT; ++q) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < RP; ++r) mx = fmaxf(mx, fmaf(a.beta, sc[q * RP + r], sBias[q * RP + r]));
+            sc[q] = mx;
+        }
+        if (g >= 0) {
+            float *Srow = a.S + ((long long)t * a.G + g) * a.Sstride + nt * NPT;
+#pragma unroll
+            for (int q = 0; q < NPT; ++q)
+                if (nt * NPT + q < a.n_level) Srow[q] = sc[q];
+        }
+    }
+    if (!ok) {
+        if (tid == 0) report(a.status, DEV_TIMEOUT);
+        // copies and MMAs still in flight finish before the memory goes away
+        if (!b_done) (void)mbar_wait(barB, 0);
+        if (m_pending) (void)mbar_wait(barM, phase);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_N) : "memory");
+}
+
+template <int RP>
+cudaError_t launch_sparse_rp(const zha_tree *t, const SparseArgs &sa, cudaStream_t st) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e =
+            cudaFuncSetAttribute(score_tc_sparse_kernel<RP>, cudaFuncAttributeMaxDynamicSharedMemorySize, TS_SMEM);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    Probe pr(t, ZHA_K_SCORE_TC, st);
+    score_tc_sparse_kernel<RP><<<dim3((unsigned)sa.ntiles, (unsigned)t->T), 128, TS_SMEM, st>>>(sa);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_score_tc_sparse(const zha_tree *t, int level, int G, const void *Q, const unsigned *M,
+                                   long long words, unsigned char *btiles, int *counts, int *lists, float *S,
+                                   long long Sstride, cudaStream_t st) {
+    const zha_config &c = t->cfg;
+    int RP = 1;
+    while (RP < c.R) RP <<= 1;
+    const long long n_level = t->n_nodes[level];
+    const long long ntiles = (n_level * RP + TC_N - 1) / TC_N;
+    cudaError_t e = launch_prep_keys(t, level, RP, ntiles, btiles, st);
+    if (e != cudaSuccess) return e;
+    MembersArgs m{};
+    m.M = M;
+    m.words = words;
+    m.ntiles = ntiles;
+    m.G = G;
+    m.NPT = TC_N / RP;
+    m.counts = counts;
+    m.lists = lists;
+    {
+        Probe pr(t, ZHA_K_SCORE_TC, st);
+        tc_members_kernel<<<dim3((unsigned)ntiles, (unsigned)t->T), 256, 0, st>>>(m);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    SparseArgs sa{};
+    sa.btiles = btiles;
+    sa.Q = static_cast<const __nv_bfloat16 *>(Q);
+    sa.counts = counts;
+    sa.lists = lists;
+    sa.ntiles = ntiles;
+    sa.n_level = n_level;
+    sa.G = G;
+    sa.beta = c.sharpness;
+    sa.S = S;
+    sa.Sstride = Sstride;
+    sa.status = t->d_status;
+    switch (RP) {
+        case 4: return launch_sparse_rp<4>(t, sa, st);
+        case 8: return launch_sparse_rp<8>(t, sa, st);
+        default: return launch_sparse_rp<16>(t, sa, st);
+    }
+}
+
+TcLayout tc_layout(int T, long long G, long long maxn_b, long long maxn_sparse, int R) {
     int RP = 1;
     while (RP < R) RP <<= 1;
     const long long mtiles = (G + TC_M * TC_MT - 1) / (TC_M * TC_MT) * TC_MT;
-    const long long ntiles = (max_level_nodes * RP + TC_N - 1) / TC_N;
-    return (size_t)T * mtiles * TC_ATILE + (size_t)T * ntiles * TC_BTILE;
+    const long long ntiles_b = (maxn_b * RP + TC_N - 1) / TC_N;
+    const long long ntiles_s = (maxn_sparse * RP + TC_N - 1) / TC_N;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    TcLayout L{};
+    L.a_off = 0;
+    L.b_off = up((size_t)T * mtiles * TC_ATILE);
+    L.counts_off = up(L.b_off + (size_t)T * ntiles_b * TC_BTILE);
+    L.lists_off = up(L.counts_off + (size_t)T * ntiles_s * sizeof(int));
+    L.bytes = up(L.lists_off + (size_t)T * ntiles_s * G * sizeof(int));
+    return L;
 }
 
 bool tc_applicable(const zha_tree *t, int G, const void *Q, zha_dtype q_dtype, int level) {
     return t->cfg.d == TC_K && q_dtype == ZHA_BF16 && (reinterpret_cast<uintptr_t>(Q) & 15) == 0 &&
            G >= TC_MIN_G && t->n_nodes[level] > 0 && t->n_nodes[level] <= TC_MAX_NODES;
+}
+
+bool tc_sparse_applicable(const zha_tree *t, int G, const void *Q, zha_dtype q_dtype, int level) {
+    // a B tile's nodes must lie in one 32-bit membership word: at least 4 columns per node
+    return t->cfg.d == TC_K && q_dtype == ZHA_BF16 && (reinterpret_cast<uintptr_t>(Q) & 15) == 0 &&
+           G >= TC_MIN_G && t->n_nodes[level] > TC_MAX_NODES && t->cfg.R > 2;
 }
 
 namespace {
@@ -477,32 +748,16 @@ cudaError_t launch_score_tc_queries(const zha_tree *t, const void *Q, int G, uns
     return cudaGetLastError();
 }
 
-cudaError_t launch_score_tc(const zha_tree *t, int level, int G, unsigned char *ws, float *S, long long Sstride,
-                            cudaStream_t st) {
+cudaError_t launch_score_tc(const zha_tree *t, int level, int G, unsigned char *atiles, unsigned char *btiles,
+                            float *S, long long Sstride, cudaStream_t st) {
     const zha_config &c = t->cfg;
     int RP = 1;
     while (RP < c.R) RP <<= 1;
     const long long mtiles = (G + TC_M * TC_MT - 1) / (TC_M * TC_MT) * TC_MT;
     const long long n_level = t->n_nodes[level];
     const long long ntiles = (n_level * RP + TC_N - 1) / TC_N;
-    unsigned char *atiles = ws;
-    unsigned char *btiles = ws + (size_t)t->T * mtiles * TC_ATILE;
-
-    PrepKeysArgs k{};
-    k.nodes = t->nodes[level];
-    k.node_tree = t->cap_nodes[level] * t->NF;
-    k.NF = t->NF;
-    k.R = c.R;
-    k.RP = RP;
-    k.D = c.d;
-    k.n_level = n_level;
-    k.ntiles = ntiles;
-    k.tiles = btiles;
-    const long long total = (long long)t->T * ntiles * TC_N * 16;
     {
-        Probe pr(t, ZHA_K_SCORE_TC, st);
-        tc_prep_keys_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(k, total);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_prep_keys(t, level, RP, ntiles, btiles, st);
         if (e != cudaSuccess) return e;
     }
 
