@@ -353,6 +353,21 @@ constexpr int HCOPIES = 8;
 constexpr float COARSE_PER_NAT = 8.f;
 constexpr int CAND_MAX = 32;  // a crossing bucket this small is resolved by one warp
 
+// Adds a fixed-point mass to a bucket kept as two 32-bit words, with native 32-bit
+// shared atomics: the low word takes the low 32 bits, and the add that wraps it
+// (old + l < old, seen in the value the atomic returns) carries one into the high
+// word, so high * 2^32 + low is the exact sum. The high word stays below 2^32 for
+// fewer than 2^24 keys (masses are at most 2^40).
+__device__ __forceinline__ void add_mass(unsigned *lo, unsigned *hi, unsigned long long v) {
+    const unsigned l = (unsigned)v;
+    unsigned h = (unsigned)(v >> 32);
+    if (l) {
+        const unsigned old = atomicAdd(lo, l);
+        h += old + l < old ? 1u : 0u;
+    }
+    if (h) atomicAdd(hi, h);
+}
+
 __device__ __forceinline__ int coarse_bucket(float s, float m) {
     const float x = (m - s) * COARSE_PER_NAT;
     return x >= 255.f ? 255 : (x > 0.f ? (int)x : 0);
@@ -366,7 +381,8 @@ template <int NT>
 __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
     chain_start();
     extern __shared__ uint32_t skey_s[];
-    __shared__ unsigned long long h_mass[HCOPIES][256];
+    // bucket masses as two 32-bit words (low word, then high word plus carries)
+    __shared__ unsigned h_mlo[HCOPIES][256], h_mhi[HCOPIES][256];
     __shared__ unsigned h_cnt[HCOPIES][256];
     __shared__ unsigned long long sh_u64[NT / 32];
     __shared__ unsigned sh_u32[NT / 32];
@@ -437,7 +453,8 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
         bool done = false;
         for (int stage = 0; stage < 6 && !done; ++stage) {
             for (int j = tid; j < HCOPIES * 256; j += NT) {
-                (&h_mass[0][0])[j] = 0;
+                (&h_mlo[0][0])[j] = 0;
+                (&h_mhi[0][0])[j] = 0;
                 (&h_cnt[0][0])[j] = 0;
             }
             if (tid == 0) s_ncand = 0;
@@ -450,7 +467,7 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
                 const int b = stage == 0 ? coarse_bucket(s, m)
                                          : (stage == 1 ? fine_bucket(s, m, cb) : (int)((k >> shift) & 255));
                 atomicAdd(&h_cnt[wcopy][b], 1u);
-                if (top_p) atomicAdd(&h_mass[wcopy][b], mass(s));
+                if (top_p) add_mass(&h_mlo[wcopy][b], &h_mhi[wcopy][b], mass(s));
             }
             __syncthreads();
             // threads 0..255 own one bucket each: buckets ascend from the highest
@@ -463,7 +480,7 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
             if (own) {
 #pragma unroll
                 for (int c = 0; c < HCOPIES; ++c) {
-                    vm += h_mass[c][b];
+                    vm += ((unsigned long long)h_mhi[c][b] << 32) + h_mlo[c][b];
                     vc += h_cnt[c][b];
                 }
             }
