@@ -71,6 +71,53 @@ __device__ __forceinline__ V block_incl_scan(V x, V *sh, V *total) {
     return base + inc;
 }
 
+// Inclusive scans of a 64-bit and a 32-bit value across a block of NT threads in
+// one pass (one set of barriers; the two shuffle chains overlap). `shm` and `shc`
+// hold NT / 32 values each; `total_m` gets the block's sum of m.
+template <int NT>
+__device__ __forceinline__ void block_incl_scan_mc(unsigned long long &m, unsigned &c, unsigned long long *shm,
+                                                   unsigned *shc, unsigned long long *total_m) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long ym = __shfl_up_sync(FULL, m, o);
+        const unsigned yc = __shfl_up_sync(FULL, c, o);
+        if (lane >= o) {
+            m += ym;
+            c += yc;
+        }
+    }
+    if (lane == 31) {
+        shm[w] = m;
+        shc[w] = c;
+    }
+    __syncthreads();
+    if (w == 0) {
+        unsigned long long x = lane < NT / 32 ? shm[lane] : 0ull;
+        unsigned y = lane < NT / 32 ? shc[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long yx = __shfl_up_sync(FULL, x, o);
+            const unsigned yy = __shfl_up_sync(FULL, y, o);
+            if (lane >= o) {
+                x += yx;
+                y += yy;
+            }
+        }
+        if (lane < NT / 32) {
+            shm[lane] = x;
+            shc[lane] = y;
+        }
+    }
+    __syncthreads();
+    if (w > 0) {
+        m += shm[w - 1];
+        c += shc[w - 1];
+    }
+    *total_m = shm[NT / 32 - 1];
+    __syncthreads();
+}
+
 template <int EPL>
 __device__ __forceinline__ void load_q(const float *p, float (&v)[EPL]) {
     if constexpr (EPL == 2) {
@@ -387,6 +434,7 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
     __shared__ unsigned long long sh_u64[NT / 32];
     __shared__ unsigned sh_u32[NT / 32];
     __shared__ uint32_t s_cand[CAND_MAX];
+    __shared__ unsigned long long s_candm[CAND_MAX];
     __shared__ int s_bucket;
     __shared__ uint32_t s_key;
     __shared__ unsigned long long s_trem;
@@ -403,27 +451,23 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
     auto key_at = [&](long long i) -> uint32_t { return skey[i]; };
 
     // stage the frontier's keys (coalesced, strided) and find the largest
+    // (batches of 8 strided positions, the last one predicated, so a thread's
+    // parent and score loads are all in flight together)
     uint32_t kmax = 0;
-    {
-        long long i = tid;
-        for (; i + 7 * NT < F; i += 8 * NT) {
-            long long id[8];
+    for (long long i = tid; i < F; i += 8 * NT) {
+        long long id[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) id[u] = frontier_id(a, par, npar, i + u * NT);
-            float v[8];
+        for (int u = 0; u < 8; ++u) id[u] = i + u * NT < F ? frontier_id(a, par, npar, i + u * NT) : -1;
+        float v[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = S[id[u]];
+        for (int u = 0; u < 8; ++u) v[u] = id[u] >= 0 ? S[id[u]] : 0.f;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 8; ++u) {
+            if (id[u] >= 0) {
                 const uint32_t k = order_key(v[u]);
                 skey[i + u * NT] = k;
                 kmax = max(kmax, k);
             }
-        }
-        for (; i < F; i += NT) {
-            const uint32_t k = order_key(S[frontier_id(a, par, npar, i)]);
-            skey[i] = k;
-            kmax = max(kmax, k);
         }
     }
     kmax = block_max_u32<NT>(kmax, sh_u32);
@@ -485,8 +529,9 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
                 }
             }
             unsigned long long total_m;
-            const unsigned long long incl_m = block_incl_scan<NT, unsigned long long>(vm, sh_u64, &total_m);
-            const unsigned incl_c = block_incl_scan<NT, unsigned>(vc, sh_u32, nullptr);
+            unsigned long long incl_m = vm;
+            unsigned incl_c = vc;
+            block_incl_scan_mc<NT>(incl_m, incl_c, sh_u64, sh_u32, &total_m);
             if (stage == 0 && top_p) {
                 trem = (unsigned long long)ceil((double)a.p * (double)total_m);
                 if (trem < 1) trem = 1;
@@ -529,18 +574,20 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
                     const bool v = lane < n;
                     const uint32_t kj = v ? s_cand[lane] : 0u;
                     const unsigned long long uj = v ? (top_p ? mass(key_to_float(kj)) : 1ull) : 0ull;
+                    s_candm[lane] = uj;
+                    __syncwarp();
+                    // every lane reads every candidate (broadcast loads, independent
+                    // of one another, so they overlap)
                     unsigned long long above = 0, same = 0;
                     unsigned same_n = 0;
-#pragma unroll
-                    for (int i = 0; i < CAND_MAX; ++i) {
-                        const uint32_t ki = __shfl_sync(FULL, kj, i);
-                        const unsigned long long ui = __shfl_sync(FULL, uj, i);
-                        if (i < n) {
-                            if (ki > kj) above += ui;
-                            else if (ki == kj) {
-                                same += ui;
-                                ++same_n;
-                            }
+#pragma unroll 8
+                    for (int i = 0; i < n; ++i) {
+                        const uint32_t ki = s_cand[i];
+                        const unsigned long long ui = s_candm[i];
+                        if (ki > kj) above += ui;
+                        else if (ki == kj) {
+                            same += ui;
+                            ++same_n;
                         }
                     }
                     const unsigned long long target = top_p ? trem : (unsigned long long)krem;
