@@ -9,10 +9,13 @@
 //   out = sum_i softmax_i(beta <q, k_i>) v_i,   lse = logsumexp_i(beta <q, k_i>).
 //
 // Design (split-K decode attention, fp32 accumulation):
-//   plan          sum the walks' key counts, set the item length from that total
-//                 so that the whole call has at most ITEM_BUDGET items (never
-//                 fewer than SEG_MIN keys each, never more than MAX_SPLIT items
-//                 per walk), and scan the walks' item and group counts into
+//   plan          sum the walks' key counts and set the item length from that
+//                 total: small calls get about as many items as the item kernel
+//                 has resident warps beyond one per walk (the per-walk rounding),
+//                 so every item starts at once, with SEG_MIN..SEG_MAX keys each;
+//                 no call has more than ITEM_BUDGET items (before per-walk
+//                 rounding) or a walk more than MAX_SPLIT; then scan the walks'
+//                 item and group counts into
 //                 offsets. Walks without keys get out = 0, lse = -inf here. Calls
 //                 of up to LOCAL_MAX_W walks plan inside every CTA of
 //                 attend_items (shared memory; a warp finds its item's walk by
@@ -40,7 +43,8 @@
 namespace zha {
 namespace {
 
-constexpr int SEG_MIN = 128;         // keys per work item, at least
+constexpr int SEG_MIN = 32;          // keys per work item, at least
+constexpr int SEG_MAX = 128;         // keys per item that small calls aim at, at most
 constexpr int MAX_SPLIT = 512;       // work items per walk, at most
 constexpr int ITEM_BUDGET = 16384;   // work items per call (before per-walk rounding)
 constexpr int GROUP = 16;            // items merged together first
@@ -51,6 +55,16 @@ __device__ __forceinline__ long long walk_keys(const int *sel_count, long long w
     int c = sel_count[w];
     c = c < 0 ? 0 : (c > max_sel ? max_sel : c);
     return (long long)C * c + tail;
+}
+
+// Keys per item of a call of `keys` keys in all: enough items to fill `target`
+// warps (SEG_MIN..SEG_MAX keys each; SEG_MAX when there is no target), and never
+// more than ITEM_BUDGET items.
+__device__ __forceinline__ long long item_length(long long keys, long long target) {
+    long long seg = target > 0 ? (keys + target - 1) / target : SEG_MAX;
+    seg = seg < SEG_MIN ? SEG_MIN : (seg > SEG_MAX ? SEG_MAX : seg);
+    const long long floor_len = (keys + ITEM_BUDGET - 1) / ITEM_BUDGET;
+    return seg > floor_len ? seg : floor_len;
 }
 
 // Keys per item of a walk of L keys, given the call's item length.
@@ -68,6 +82,7 @@ struct PlanArgs {
     const int *sel_count;
     int max_sel, C, D, out_bf16;
     long long tail, W;
+    long long target_items;  // resident item warps beyond one per walk (0: none)
     int *item_off;    // [W + 1]
     int *group_off;   // [W + 1]
     int *seg;         // [1] keys per item of the call (before the per-walk cap)
@@ -130,8 +145,7 @@ __global__ void __launch_bounds__(1024) attend_plan_kernel(PlanArgs a) {
         block_scan2(keys, zero, sh, total, unused);
         keys = total;
     }
-    long long seg = (keys + ITEM_BUDGET - 1) / ITEM_BUDGET;
-    if (seg < SEG_MIN) seg = SEG_MIN;
+    long long seg = item_length(keys, a.target_items);
     if (seg > (1LL << 30)) seg = 1LL << 30;
     if (threadIdx.x == 0) a.seg[0] = (int)seg;
 
@@ -181,6 +195,7 @@ struct ItemArgs {
     int max_sel, C, G, D;
     int c_shift;  // log2(C) when C is a power of two, else -1
     long long W, cap, n1, tail;
+    long long target_items;  // as in PlanArgs
     float beta;
     float *partial;   // [items][D + 4]: acc[D], m, l (rows 16-byte aligned)
     float *gpartial;  // [groups][D + 4]: the same, per group
@@ -307,8 +322,7 @@ __device__ long long local_plan(const ItemArgs &a, int *s_io, int *s_go, int *s_
     }
     long long zero = 0, total_keys, unused;
     block_scan2(keys, zero, sh, total_keys, unused);
-    long long seg = (total_keys + ITEM_BUDGET - 1) / ITEM_BUDGET;
-    if (seg < SEG_MIN) seg = SEG_MIN;
+    long long seg = item_length(total_keys, a.target_items);
     if (seg > (1LL << 30)) seg = 1LL << 30;
     long long ni = 0, ng = 0;
     for (int w = w0; w < w1; ++w) {
@@ -589,16 +603,23 @@ __global__ void __launch_bounds__(256) attend_items_kernel(ItemArgs a) {
     chain_done();
 }
 
+// Resident CTAs of the item kernel per SM (computed once).
 template <typename T, int D, bool LOCAL>
-cudaError_t launch_items(const zha_tree *t, const ItemArgs &ia, long long max_items, cudaStream_t st) {
+int items_per_sm() {
     static int per_sm = 0;
-    const size_t smem = LOCAL ? sizeof(int) * (3 * (size_t)ia.W + 2) : 0;
     if (!per_sm) {
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attend_items_kernel<T, D, LOCAL>, 256,
                                                           sizeof(int) * (3 * LOCAL_MAX_W + 2)) != cudaSuccess ||
             per_sm < 1)
             per_sm = 1;
     }
+    return per_sm;
+}
+
+template <typename T, int D, bool LOCAL>
+cudaError_t launch_items(const zha_tree *t, const ItemArgs &ia, long long max_items, cudaStream_t st) {
+    const int per_sm = items_per_sm<T, D, LOCAL>();
+    const size_t smem = LOCAL ? sizeof(int) * (3 * (size_t)ia.W + 2) : 0;
     long long blocks = (max_items + 7) / 8;
     const long long cap = (long long)num_sms() * per_sm;
     if (blocks > cap) blocks = cap;
@@ -611,6 +632,21 @@ template <typename T, int D>
 cudaError_t launch_items_any(const zha_tree *t, const ItemArgs &ia, long long max_items, cudaStream_t st) {
     return ia.W <= LOCAL_MAX_W ? launch_items<T, D, true>(t, ia, max_items, st)
                                : launch_items<T, D, false>(t, ia, max_items, st);
+}
+
+// Warps of the item kernel resident at once (its grid never exceeds them).
+template <typename T, int D>
+long long resident_item_warps(long long W) {
+    const int per_sm = W <= LOCAL_MAX_W ? items_per_sm<T, D, true>() : items_per_sm<T, D, false>();
+    return (long long)num_sms() * per_sm * 8;
+}
+long long resident_item_warps(zha_dtype kv, int D, long long W) {
+    const bool bf = kv == ZHA_BF16;
+    switch (D) {
+        case 64: return bf ? resident_item_warps<__nv_bfloat16, 64>(W) : resident_item_warps<float, 64>(W);
+        case 128: return bf ? resident_item_warps<__nv_bfloat16, 128>(W) : resident_item_warps<float, 128>(W);
+        default: return bf ? resident_item_warps<__nv_bfloat16, 256>(W) : resident_item_warps<float, 256>(W);
+    }
 }
 
 }  // namespace
@@ -690,6 +726,12 @@ cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zh
     pl.group_done = s.group_done;
     pl.out = out;
     pl.lse = lse;
+    // small calls: one item per resident warp, less one per walk for the rounding
+    // of each walk's keys into items
+    {
+        const long long target = resident_item_warps(c.kv_dtype, c.d, W) - W;
+        pl.target_items = target > 0 ? target : 0;
+    }
     if (W <= LOCAL_MAX_W) {
         // the item kernel plans for itself; only the completion counters (walk
         // and group tickets, adjacent in the scratch) must start at zero
@@ -725,6 +767,7 @@ cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zh
     ia.cap = c.capacity;
     ia.n1 = t->n_nodes[1];
     ia.tail = pl.tail;
+    ia.target_items = pl.target_items;
     ia.beta = c.sharpness;
     ia.partial = s.partial;
     ia.gpartial = s.gpartial;
