@@ -15,11 +15,11 @@
 //                 so every item starts at once, with SEG_MIN..SEG_MAX keys each;
 //                 no call has more than ITEM_BUDGET items (before per-walk
 //                 rounding) or a walk more than MAX_SPLIT; then scan the walks'
-//                 item and group counts into
-//                 offsets. Walks without keys get out = 0, lse = -inf here. Calls
-//                 of up to LOCAL_MAX_W walks plan inside every CTA of
-//                 attend_items (shared memory; a warp finds its item's walk by
-//                 binary search) after a memset clears the completion counters;
+//                 item and group counts into offsets. Walks without keys get
+//                 out = 0, lse = -inf here. Calls of up to LOCAL_MAX_W walks plan
+//                 inside every CTA of attend_items (shared memory; a warp finds
+//                 its item's walk by binary search) after a small clear kernel
+//                 zeroes the completion counters;
 //                 larger calls run attend_plan (one CTA) first, which also writes
 //                 an item -> walk map and clears the counters.
 //   attend_items  grid-stride over items, one warp per item. The item's chunk
