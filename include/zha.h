@@ -70,7 +70,8 @@ typedef struct {
     int d;              /* head dimension: 64, 128 or 256 */
     int R;              /* reference queries per tree, 1..16 */
     int chunk;          /* C: children per node, 2..64 */
-    int depth;          /* levels built, 1..ZHA_MAX_DEPTH */
+    int depth;          /* levels built, 1..ZHA_MAX_DEPTH; or 0: grow with the keys
+                           (see zha_build) */
     int top_width;      /* a walk starts at the lowest level holding at most this
                            many nodes (the deepest level if none does); >= 1.
                            [P1] "Run a small tree yourself": the demo's top level
@@ -116,6 +117,13 @@ typedef struct zha_tree zha_tree;
  * Node storage is allocated here for `capacity` keys: level l holds
  * floor(capacity / C^l) nodes of R*d + round_up(R, 4) fp32 each (keys [R][d],
  * then biases [R], then padding).
+ * Depth. With cfg->depth >= 1 the tree has exactly that many levels. With
+ * cfg->depth == 0 its depth grows with the keys ([P4], abstract: the depth of
+ * the tree of summaries grows with the context): the tree has every level that
+ * holds at least one node, D = max(1, floor(log_C n)) levels, at most
+ * ZHA_MAX_DEPTH and at most the levels `capacity` can fill (storage for those
+ * is allocated here). An append that completes a group of C nodes at the top
+ * level makes their parent and so starts level D + 1. zha_depth returns D.
  * Errors: ZHA_ERR_INVALID (NULL pointer, shape out of range, n_keys > capacity),
  * ZHA_ERR_OOM, ZHA_ERR_CUDA.
  */
@@ -126,8 +134,10 @@ int zha_build(const zha_config *cfg, void *K, void *V, const float *refs, long l
  * zha_append: append one key and one value to every tree at position n (the
  * current key count), then make the nodes whose chunk this fills: the level-1
  * node if (n+1) % C == 0, its parent if that completes a group of C at level 1,
- * and so on up to `depth`. [P1] "How is the tree built?": a node is created each
- * time a chunk fills. The result equals zha_build over the n+1 keys.
+ * and so on up to `depth` (for a growing tree, up to the deepest level its
+ * capacity allows, which raises the depth when a new top node is made). [P1]
+ * "How is the tree built?": a node is created each time a chunk fills. The
+ * result equals zha_build over the n+1 keys.
  * k_new, v_new: [B][H_kv][d] of kv_dtype (device).
  * Errors: ZHA_ERR_INVALID (NULL), ZHA_ERR_CAPACITY (n == capacity), ZHA_ERR_CUDA.
  */
@@ -263,6 +273,10 @@ int zha_last_search_info(zha_tree *tree, zha_search_info *out, void *stream);
 
 /* Keys currently in every tree (n). */
 long long zha_num_keys(const zha_tree *tree);
+
+/* Levels the trees currently have (cfg->depth, or for a growing tree the
+   deepest level holding a node, at least 1); -1 for a NULL handle. */
+int zha_depth(const zha_tree *tree);
 
 /* Waits for the tree's pending work on `stream`, then returns and clears the
    first device-side error recorded since the last call (ZHA_OK if none). */

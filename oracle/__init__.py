@@ -10,7 +10,11 @@ marshals numpy arrays and keeps the per-level arrays of one tree. The tree
 shape follows page "How does a tree of summaries search a context? How ZHA
 works", sections "How is the tree built?" and "Run a small tree yourself":
 level l has floor(n_{l-1} / C) nodes, node j summarizing nodes C*j .. C*j+C-1
-of level l-1, and a node is made when its chunk fills.
+of level l-1, and a node is made when its chunk fills. A tree built with depth 0
+grows its depth with the keys (page "Subquadratic Attention with a Hierarchical
+Tree-Structured Indexer", abstract: the tree's depth grows with the context): it
+keeps every level that holds a node, and the parent made when a group of C top
+nodes fills starts a new level.
 """
 from __future__ import annotations
 
@@ -151,6 +155,8 @@ class Tree:
     n_nodes: list = field(default_factory=list)
     keys: list = field(default_factory=list)
     bias: list = field(default_factory=list)
+    grow: bool = False  # depth follows the key count
+    max_depth: int = 0  # levels with storage (depth unless the tree grows)
 
     @property
     def n_keys(self) -> int:
@@ -164,7 +170,7 @@ class Tree:
 def _alloc_tree(capacity: int, refs, C: int, depth: int, beta: float, store: int) -> Tree:
     refs = _f64(refs)
     R, d = refs.shape
-    t = Tree(C=C, depth=depth, beta=float(beta), R=R, d=d, store=store, refs=refs)
+    t = Tree(C=C, depth=depth, beta=float(beta), R=R, d=d, store=store, refs=refs, max_depth=depth)
     t.n_nodes = [0] * (depth + 1)
     t.keys = [None] * (depth + 1)
     t.bias = [None] * (depth + 1)
@@ -189,25 +195,48 @@ def _build_nodes(t: Tree, K: np.ndarray, l: int, begin: int, end: int, threads: 
                                     threads), f"level-{l} build")
 
 
+def levels_filled(count: int, C: int, limit: int = MAX_LEVELS - 1) -> int:
+    """The number of levels ``count`` keys fill with at least one node each (at
+    least 1, at most ``limit``)."""
+    levels, n = 0, count
+    while levels < limit:
+        n //= C
+        if n < 1:
+            break
+        levels += 1
+    return max(levels, 1)
+
+
 def build_tree(K, refs, C: int, depth: int, beta: float, store: int = STORE_F32,
-               threads: int = 0, capacity: int | None = None) -> Tree:
-    """Build every level of the tree over the keys ``K`` [N][d] (exact doubles)."""
+               threads: int = 0, capacity: int | None = None, max_levels: int = MAX_LEVELS - 1) -> Tree:
+    """Build every level of the tree over the keys ``K`` [N][d] (exact doubles).
+    depth >= 1: that many levels. depth == 0: the depth grows with the keys, every
+    level holding a node is kept (at most ``max_levels``), with storage for every
+    level the capacity can fill."""
     K = _f64(K)
     N = K.shape[0]
-    t = _alloc_tree(max(N, capacity or 0), refs, C, depth, beta, store)
+    cap = max(N, capacity or 0)
+    grow = depth == 0
+    levels = levels_filled(cap, C, max_levels) if grow else depth
+    t = _alloc_tree(cap, refs, C, levels, beta, store)
+    t.grow = grow
     t.n_nodes[0] = N
     n = N
-    for l in range(1, depth + 1):
+    for l in range(1, levels + 1):
         n //= C
         t.n_nodes[l] = n
         _build_nodes(t, K, l, 0, n, threads)
+    if grow:
+        t.depth = max([1] + [l for l in range(1, levels + 1) if t.n_nodes[l] > 0])
     return t
 
 
 def append(t: Tree, K_all, count: int, threads: int = 0) -> None:
     """Append ``count`` keys one at a time (the keys are ``K_all[n0 : n0+count]``,
     where n0 is the current key count). Each time a chunk fills, its level-1 node is
-    made; each time a group of C nodes fills at level l < depth, its parent is made."""
+    made; each time a group of C nodes fills at level l < depth, its parent is made
+    (for a growing tree, up to the deepest level with storage: the parent of a full
+    top group starts a new level)."""
     K = _f64(K_all)
     for _ in range(count):
         n0 = t.n_nodes[0] + 1
@@ -215,7 +244,7 @@ def append(t: Tree, K_all, count: int, threads: int = 0) -> None:
             raise ValueError("append past the keys provided")
         t.n_nodes[0] = n0
         below = n0
-        for l in range(1, t.depth + 1):
+        for l in range(1, t.max_depth + 1):
             if below % t.C != 0:
                 break
             j = below // t.C - 1
@@ -223,6 +252,8 @@ def append(t: Tree, K_all, count: int, threads: int = 0) -> None:
                 raise ValueError("append past the tree's capacity")
             _build_nodes(t, K, l, j, j + 1, threads)
             t.n_nodes[l] = j + 1
+            if l > t.depth:
+                t.depth = l
             below = j + 1
 
 

@@ -61,6 +61,10 @@ def test_host_side_argument_checks(zha):
     cfg.chunk = 1
     assert L.zha_build(ctypes.byref(cfg), None, None, None, 0, None, ctypes.byref(h)) == zha.ERR_INVALID
     cfg.chunk = 4
+    cfg.depth = -1
+    assert L.zha_build(ctypes.byref(cfg), None, None, None, 0, None, ctypes.byref(h)) == zha.ERR_INVALID
+    assert b"depth" in L.zha_last_error()
+    cfg.depth = 0  # a growing tree: the config is valid, the NULL pointers are not
     assert L.zha_build(ctypes.byref(cfg), None, None, None, 0, None, ctypes.byref(h)) == zha.ERR_INVALID
     assert b"NULL" in L.zha_last_error()
     assert h.value is None
@@ -71,6 +75,7 @@ def test_host_side_argument_checks(zha):
     assert L.zha_reserve(None, 1, 1) == zha.ERR_INVALID
     assert L.zha_dense_scan(None, None, 0, 1, 1, 0, 0.9, 1, None, None, 1, None) == zha.ERR_INVALID
     assert L.zha_num_keys(None) == -1
+    assert L.zha_depth(None) == -1
     assert L.zha_sync_status(None, None) == zha.ERR_INVALID
     L.zha_destroy(None)
 

@@ -202,10 +202,12 @@ def _check_against_oracle(K, V, refs, Q, N, C, depth, beta, top_width=64, modes=
     group = Hq // H
     R = refs.shape[1]
     Qh = host64(Q)
+    levels = tree.depth  # depth 0: the levels the keys fill, on both sides
     for b in range(B):
         for h in range(H):
             ot = O.build_tree(host64(K[b, h, :N]), host64(refs[h]), C, depth, beta, store=O.STORE_F32)
-            for l in range(1, depth + 1):
+            assert ot.depth == levels
+            for l in range(1, levels + 1):
                 g, n = gpu_level(tree, l, b * H + h)
                 assert n == ot.n_nodes[l]
                 if n:
@@ -333,6 +335,45 @@ def test_append_equals_build():
             assert_nodes_close(g, *ot.level(l), R, d)
     grown.close()
     direct.close()
+
+
+def test_growing_depth():
+    """depth 0: the trees keep every level that holds a node, and the append that
+    completes a full group of C top nodes starts a new level. The grown trees
+    equal a growing build over the final keys bit for bit, and the oracle."""
+    Z = zha()
+    B, H, d, R, C = 2, 2, 128, 8, 4
+    N0, M = 250, 30
+    K, V, refs, Q = _tiny(N0 + M, C=C, d=d, R=R, B=B, H=H, Hq=4, nq=3, dtype=torch.bfloat16, seed=5)
+    beta = 1 / np.sqrt(d)
+    grown_K, grown_V = K.clone(), V.clone()
+    grown_K[:, :, N0:] = 0
+    grown_V[:, :, N0:] = 0
+    grown = Z.Tree(grown_K, grown_V, refs, N0, C, 0, beta)
+    # 250 keys: 62, 15, 3 nodes; the 256th key (4^4) completes a group at every level
+    assert grown.depth == 3 and grown.level_sizes() == [250, 62, 15, 3]
+    for i in range(N0, N0 + M):
+        grown.append(K[:, :, i].contiguous(), V[:, :, i].contiguous())
+        assert grown.depth == (4 if i + 1 >= 256 else 3), i
+    direct = Z.Tree(K, V, refs, N0 + M, C, 0, beta)
+    assert direct.depth == 4
+    assert grown.level_sizes() == direct.level_sizes() == [280, 70, 17, 4, 1]
+    for l in range(1, 5):
+        a, n = grown.level(l)
+        b, m = direct.level(l)
+        assert torch.equal(a[:, :n], b[:, :m])  # same kernel, same inputs: bit-identical
+    ot = O.build_tree(host64(K[1, 0, :N0]), host64(refs[0]), C, 0, beta, capacity=N0 + M)
+    O.append(ot, host64(K[1, 0]), M)
+    assert ot.depth == 4
+    for l in range(1, 5):
+        g, n = gpu_level(grown, l, 2)
+        assert n == ot.n_nodes[l]
+        assert_nodes_close(g, *ot.level(l), R, d)
+    grown.close()
+    direct.close()
+    # search and attention on a growing tree against the oracle
+    _check_against_oracle(K, V, refs, Q, N0 + M, C, 0, beta, top_width=2,
+                          modes=((O.TOP_P, 0.9, 0), (O.TOP_K, 0, 3)))
 
 
 def test_append_past_capacity_is_refused():

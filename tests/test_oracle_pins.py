@@ -292,6 +292,62 @@ def test_append_equals_build():
         assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
+# Depths worked by hand: 4096 = 4^6 keys fill 6 levels; 4095 stop one short
+# (1023, 255, 63, 15, 3, then 0); 7 keys fill no chunk of 8 (one empty level);
+# 100 keys with C = 8 give 12 and 1; 1003 give 125, 15, 1; 250 with C = 2 give
+# 125, 62, 31, 15, 7, 3, 1.
+@pytest.mark.parametrize("N,C,D", [(4096, 4, 6), (4095, 4, 5), (7, 8, 1), (100, 8, 2), (1003, 8, 3), (250, 2, 7)])
+def test_growing_tree_keeps_every_filled_level(N, C, D):
+    d, R = 8, 2
+    rng = np.random.default_rng(N + C)
+    K = rng.standard_normal((N, d))
+    refs = rng.standard_normal((R, d))
+    t = O.build_tree(K, refs, C, 0, 0.5)
+    assert t.grow and t.depth == D
+    # the top level holds a node (when any chunk is full) but never a full group
+    # of C, which would have a parent one level up
+    assert (t.n_nodes[D] >= 1) == (N >= C)
+    assert t.n_nodes[D] < C
+    # it is the fixed-depth tree of D levels, walks included
+    fixed = O.build_tree(K, refs, C, D, 0.5)
+    for l in range(1, D + 1):
+        a, b = t.level(l), fixed.level(l)
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    for qi in range(3):
+        q = rng.standard_normal(d)
+        w, v = O.search(t, q, O.TOP_P, 0.9, 0, top_width=4), O.search(fixed, q, O.TOP_P, 0.9, 0, top_width=4)
+        assert list(w.sel) == list(v.sel) and w.start_level == v.start_level
+
+
+def test_append_grows_the_depth_at_a_full_top_group():
+    # C = 4: 60 keys give 15 and 3 nodes (depth 2); the 64th key completes the 16th
+    # level-1 node, which completes the 4th level-2 node, whose group of 4 gets a
+    # parent: depth 3
+    d, R, C = 8, 3, 4
+    rng = np.random.default_rng(11)
+    K = rng.standard_normal((80, d)).astype(np.float32).astype(np.float64)
+    refs = rng.standard_normal((R, d))
+    grown = O.build_tree(K[:60], refs, C, 0, 0.4, capacity=80)
+    assert grown.depth == 2 and grown.max_depth == 3
+    O.append(grown, K, 3)
+    assert grown.depth == 2 and grown.n_nodes == [63, 15, 3, 0]
+    O.append(grown, K, 1)
+    assert grown.depth == 3 and grown.n_nodes == [64, 16, 4, 1]
+    direct = O.build_tree(K[:64], refs, C, 0, 0.4, capacity=80)
+    assert direct.depth == 3 and direct.n_nodes == grown.n_nodes
+    for l in range(1, 4):
+        a, b = grown.level(l), direct.level(l)
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    for qi in range(4):
+        q = rng.standard_normal(d) * 2
+        for mode, p, k in [(O.TOP_P, 0.9, 0), (O.TOP_K, 0, 3)]:
+            w = O.search(grown, q, mode, p, k, top_width=2)
+            assert w.start_level == 3
+            if min(w.tie_gap, w.tie_sum) < 1e-12:
+                continue
+            assert list(w.sel) == _brute_walk(grown, q, mode, p, k, 2)
+
+
 def test_attend_on_a_subset_is_softmax_attention():
     rng = np.random.default_rng(10)
     N, d, C = 333, 12, 4

@@ -26,7 +26,7 @@ TOP_P, TOP_K = 0, 1
 
 # Every symbol include/zha.h declares.
 SYMBOLS = ("zha_build", "zha_append", "zha_search", "zha_attend", "zha_reserve", "zha_level",
-           "zha_num_keys", "zha_sync_status", "zha_destroy", "zha_last_error", "zha_version",
+           "zha_num_keys", "zha_depth", "zha_sync_status", "zha_destroy", "zha_last_error", "zha_version",
            "zha_profile", "zha_profile_read", "zha_kernel_launches", "zha_last_search_info",
            "zha_dense_scan", "zha_attend_noalloc")
 KERNEL_KINDS = ("build", "append", "search_init", "score", "select", "attend_plan", "attend_partial",
@@ -85,6 +85,8 @@ def lib():
                                 ctypes.POINTER(i)]
         L.zha_num_keys.argtypes = [vp]
         L.zha_num_keys.restype = ll
+        L.zha_depth.argtypes = [vp]
+        L.zha_depth.restype = ctypes.c_int
         L.zha_sync_status.argtypes = [vp, vp]
         L.zha_destroy.argtypes = [vp]
         L.zha_destroy.restype = None
@@ -166,9 +168,15 @@ class Tree:
     def n_keys(self) -> int:
         return int(lib().zha_num_keys(self._h))
 
+    @property
+    def depth(self) -> int:
+        """Levels the trees have now (the configured depth, or for depth=0 the
+        deepest level holding a node)."""
+        return int(lib().zha_depth(self._h))
+
     def level_sizes(self) -> list:
         out = [self.n_keys]
-        for l in range(1, self.cfg.depth + 1):
+        for l in range(1, self.depth + 1):
             out.append(self.level(l)[1])
         return out
 

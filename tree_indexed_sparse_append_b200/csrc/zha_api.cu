@@ -44,7 +44,8 @@ int check_config(const zha_config *c) {
     if (c->d != 64 && c->d != 128 && c->d != 256) return fail(ZHA_ERR_INVALID, "d must be 64, 128 or 256 (got %d)", c->d);
     if (c->R < 1 || c->R > 16) return fail(ZHA_ERR_INVALID, "R must be in 1..16 (got %d)", c->R);
     if (c->chunk < 2 || c->chunk > 64) return fail(ZHA_ERR_INVALID, "chunk must be in 2..64 (got %d)", c->chunk);
-    if (c->depth < 1 || c->depth > ZHA_MAX_DEPTH) return fail(ZHA_ERR_INVALID, "depth must be in 1..%d", ZHA_MAX_DEPTH);
+    if (c->depth < 0 || c->depth > ZHA_MAX_DEPTH)
+        return fail(ZHA_ERR_INVALID, "depth must be in 1..%d, or 0 to grow with the keys", ZHA_MAX_DEPTH);
     if (c->top_width < 1) return fail(ZHA_ERR_INVALID, "top_width must be >= 1");
     if (c->capacity < 1) return fail(ZHA_ERR_INVALID, "capacity must be >= 1");
     if (c->capacity > (1LL << 31) - 1) return fail(ZHA_ERR_INVALID, "capacity must fit in int32 key ids");
@@ -59,11 +60,19 @@ int start_level(const zha_tree *t) {
     return t->cfg.depth;
 }
 
+// Live node counts of every level with storage; a growing tree's depth is then
+// its deepest level holding a node (at least 1).
 void set_counts(zha_tree *t) {
     long long n = t->n;
-    for (int l = 1; l <= t->cfg.depth; ++l) {
+    for (int l = 1; l <= t->max_depth; ++l) {
         n /= t->cfg.chunk;
         t->n_nodes[l] = n;
+    }
+    if (t->grow) {
+        int d = 1;
+        for (int l = 2; l <= t->max_depth; ++l)
+            if (t->n_nodes[l] > 0) d = l;
+        t->cfg.depth = d;
     }
 }
 
@@ -140,7 +149,7 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     const long long W = walks < 1 ? 1 : walks;
     (void)max_sel;  // the layout depends on the walks and the tree only
     const long long cap1 = t->cap_nodes[1] > 0 ? t->cap_nodes[1] : 1;
-    const long long cap2 = c.depth >= 2 && t->cap_nodes[2] > 0 ? t->cap_nodes[2] : 1;
+    const long long cap2 = t->max_depth >= 2 && t->cap_nodes[2] > 0 ? t->cap_nodes[2] : 1;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         size_t o = off;
@@ -157,10 +166,11 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     size_t o_M[ZHA_MAX_DEPTH + 1] = {0}, o_U[ZHA_MAX_DEPTH + 1] = {0};
     // membership bits: per level, [T][words][G] with T * G = W
     const size_t M_start = off;
-    for (int l = 1; l <= c.depth; ++l) o_M[l] = take(sizeof(unsigned) * W * ((t->cap_nodes[l] + 31) / 32));
+    // (every level with storage: a growing tree may deepen after this reservation)
+    for (int l = 1; l <= t->max_depth; ++l) o_M[l] = take(sizeof(unsigned) * W * ((t->cap_nodes[l] + 31) / 32));
     const size_t M_bytes = off - M_start;
     const size_t U_start = off;
-    for (int l = 1; l <= c.depth; ++l) o_U[l] = take(sizeof(unsigned) * t->T * ((t->cap_nodes[l] + 31) / 32));
+    for (int l = 1; l <= t->max_depth; ++l) o_U[l] = take(sizeof(unsigned) * t->T * ((t->cap_nodes[l] + 31) / 32));
     const size_t U_bytes = off - U_start;
     const AttendLayout att = attend_layout(W, c.d);
     const size_t o_att = take(att.bytes);
@@ -169,7 +179,7 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     TcLayout tcl{};
     if (c.d == 128 && Gw >= TC_MIN_G) {
         long long maxn_b = 0, maxn_sparse = 0;
-        for (int l = 1; l <= c.depth; ++l) {
+        for (int l = 1; l <= t->max_depth; ++l) {
             maxn_b = std::max(maxn_b, t->cap_nodes[l]);
             if (t->cap_nodes[l] > TC_MAX_NODES) maxn_sparse = std::max(maxn_sparse, t->cap_nodes[l]);
         }
@@ -198,8 +208,8 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     s->cnt[0] = reinterpret_cast<int *>(b + o_c0);
     s->cnt[1] = reinterpret_cast<int *>(b + o_c1);
     for (int l = 0; l <= ZHA_MAX_DEPTH; ++l) {
-        s->M[l] = l >= 1 && l <= c.depth ? reinterpret_cast<unsigned *>(b + o_M[l]) : nullptr;
-        s->U[l] = l >= 1 && l <= c.depth ? reinterpret_cast<unsigned *>(b + o_U[l]) : nullptr;
+        s->M[l] = l >= 1 && l <= t->max_depth ? reinterpret_cast<unsigned *>(b + o_M[l]) : nullptr;
+        s->U[l] = l >= 1 && l <= t->max_depth ? reinterpret_cast<unsigned *>(b + o_U[l]) : nullptr;
     }
     s->M_base = reinterpret_cast<unsigned *>(b + M_start);
     s->U_base = reinterpret_cast<unsigned *>(b + U_start);
@@ -255,8 +265,20 @@ int zha_build(const zha_config *cfg, void *K, void *V, const float *refs, long l
     t->refs = refs;
     t->n = n_keys;
     cudaGetDevice(&t->device);
+    // a growing tree gets storage for every level its capacity can fill
+    t->grow = cfg->depth == 0;
+    t->max_depth = cfg->depth;
+    if (t->grow) {
+        long long c = cfg->capacity;
+        t->max_depth = 1;
+        for (int l = 1; l <= ZHA_MAX_DEPTH; ++l) {
+            c /= cfg->chunk;
+            if (c < 1) break;
+            t->max_depth = l;
+        }
+    }
     long long cap = cfg->capacity;
-    for (int l = 1; l <= cfg->depth; ++l) {
+    for (int l = 1; l <= t->max_depth; ++l) {
         cap /= cfg->chunk;
         t->cap_nodes[l] = cap;
         if (cap > 0) {
@@ -277,7 +299,8 @@ int zha_build(const zha_config *cfg, void *K, void *V, const float *refs, long l
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     e = cudaMemsetAsync(t->d_status, 0, sizeof(int), st);
     set_counts(t);
-    for (int l = 1; l <= cfg->depth && e == cudaSuccess; ++l) e = zha::launch_build_level(t, l, 0, t->n_nodes[l], st);
+    for (int l = 1; l <= t->max_depth && e == cudaSuccess; ++l)
+        e = zha::launch_build_level(t, l, 0, t->n_nodes[l], st);
     if (e != cudaSuccess) {
         zha_destroy(t);
         return cuda_fail(e, "launching the tree build");
@@ -293,11 +316,12 @@ int zha_append(zha_tree *t, const void *k_new, const void *v_new, void *stream) 
     ZHA_CUDA(zha::launch_append_kv(t, k_new, v_new, st), "launching the append");
     t->n += 1;
     long long below = t->n;
-    for (int l = 1; l <= t->cfg.depth; ++l) {
+    for (int l = 1; l <= t->max_depth; ++l) {
         if (below % t->cfg.chunk != 0) break;
         const long long j = below / t->cfg.chunk - 1;
         ZHA_CUDA(zha::launch_build_level(t, l, j, j + 1, st), "launching a node build");
         t->n_nodes[l] = j + 1;
+        if (l > t->cfg.depth) t->cfg.depth = l;  // a growing tree's first node of a new level
         below = j + 1;
     }
     return ZHA_OK;
@@ -424,6 +448,8 @@ int zha_level(const zha_tree *t, int level, const float **nodes, long long *n_no
 }
 
 long long zha_num_keys(const zha_tree *t) { return t ? t->n : -1; }
+
+int zha_depth(const zha_tree *t) { return t ? t->cfg.depth : -1; }
 
 int zha_sync_status(zha_tree *t, void *stream) {
     if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");

@@ -176,6 +176,8 @@ struct zha_tree {
     int NF;                                 // floats per node
     int device;
     long long n;                            // keys per tree
+    int max_depth;                          // levels with storage (cfg.depth unless the tree grows)
+    int grow;                               // 1: cfg.depth follows the key count
     long long n_nodes[ZHA_MAX_DEPTH + 1];   // live nodes per tree, per level
     long long cap_nodes[ZHA_MAX_DEPTH + 1]; // node capacity per tree, per level
     float *nodes[ZHA_MAX_DEPTH + 1];        // [T][cap_nodes[l]][NF]
