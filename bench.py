@@ -346,6 +346,30 @@ def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes
                             "keys_selected_mean": float(dcnt.float().mean().item()),
                             "tree_search_ms": search_ms, "dense_over_tree_search": ms / search_ms}
         del dsel, dcnt
+        # chunk-mass profile of the same dense attention: per walk, the fewest
+        # 16-key chunks holding 90% of it (the statistic the pages quote for real
+        # models at about 64K tokens; these keys are synthetic)
+        group = 16
+        n_chunks = (tree.n_keys + group - 1) // group
+        csel = torch.empty(Wk, n_chunks, dtype=torch.int32, device=dev)
+        ccnt = torch.empty(Wk, dtype=torch.int32, device=dev)
+        for _ in range(3):
+            tree.chunk_mass(inp.Q, group, 0.9, max_sel=n_chunks, out=(csel, ccnt))
+        ts = []
+        for _ in range(10):
+            flush.zero_()
+            e0.record(st)
+            tree.chunk_mass(inp.Q, group, 0.9, max_sel=n_chunks, out=(csel, ccnt))
+            e1.record(st)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        tree.sync_status()
+        share = ccnt.float() / n_chunks
+        dense["chunk_mass"] = {"group": group, "p": 0.9, "n_chunks": n_chunks, "ms": sorted(ts)[len(ts) // 2],
+                               "share_median": float(share.median().item()),
+                               "share_p10": float(share.quantile(0.1).item()),
+                               "share_p90": float(share.quantile(0.9).item())}
+        del csel, ccnt
 
     # end to end through the public API with host buffers
     mname, p, k = modes[0]

@@ -211,6 +211,27 @@ int zha_dense_scan(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_hea
                    void *stream);
 
 /*
+ * zha_chunk_mass: how concentrated each query's dense attention is over chunks of
+ * keys ([P1] "How does top-p differ from top-K?": measured at about 64K tokens,
+ * 90% of the attention sits in a median of 2.3% to 15% of the 16-key chunks,
+ * depending on the task; no counterpart in the tree walk itself). For every
+ * walk: the softmax of beta*<q, k_j> over all n keys of its tree, summed over
+ * consecutive chunks of `group` keys (the last chunk may be partial), and the
+ * fewest chunks whose summed mass reaches p, taken by mass, largest first, ties
+ * to the lower chunk index (p >= 1 takes every chunk).
+ * Q:     [B][H_q][n_q][d] of q_dtype; at most 32 walks per tree.
+ * group: keys per chunk, >= 1 (16 in the measurement quoted above).
+ * sel:   [walks][max_sel] int32: the chunk indices taken, ascending.
+ * count: [walks] int32: how many; count / ceil(n / group) is the walk's share.
+ * Scratch of 4 * walks * n + 8 * walks * ceil(n / group) bytes (+ the queries in
+ * fp32) is taken from the tree.
+ * Errors as zha_dense_scan (a walk taking more than max_sel chunks keeps the
+ * first max_sel and makes zha_sync_status return ZHA_ERR_CAPACITY).
+ */
+int zha_chunk_mass(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q, int group, float p,
+                   int *sel, int *count, int max_sel, void *stream);
+
+/*
  * zha_reserve: allocate the search and attend scratch for up to max_walks walks
  * and selections of up to max_sel chunks now, so that later calls with at most
  * these sizes allocate nothing (e.g. before capturing them in a CUDA graph).

@@ -325,6 +325,35 @@ def dense_scan(K, q, beta: float, mode: int = TOP_P, p: float = 0.9, k: int = 1)
     return sel[: n.value].copy(), tg.value, ts.value
 
 
+def chunk_mass(K, q, beta: float, group: int = 16, p: float = 0.9):
+    """How concentrated the dense attention of ``q`` is over chunks of keys (page
+    "How does a tree of summaries search a context? How ZHA works", section "How
+    does top-p differ from top-K?": the share of 16-key chunks holding 90% of the
+    attention). The softmax of beta*<q, k_j> over all keys, summed over
+    consecutive chunks of ``group`` keys (the last may be partial); the fewest
+    chunks whose masses reach ``p``, taken largest first, ties to the lower chunk
+    (every chunk when p >= 1). Returns (chunk ids ascending, number of chunks,
+    tie_gap, tie_sum): tie_gap is the relative mass gap between the last chunk
+    taken and the first left out, tie_sum the distance of the running sum before
+    or after the last chunk taken from p, relative to p."""
+    K = _f64(K)
+    q = _f64(q)
+    n = K.shape[0]
+    if n == 0:
+        return np.zeros(0, dtype=np.int64), 0, np.inf, np.inf
+    s = beta * (K @ q)
+    w = np.exp(s - s.max())
+    w /= w.sum()
+    m = np.add.reduceat(w, np.arange(0, n, group))
+    order = np.argsort(-m, kind="stable")
+    cum = np.cumsum(m[order])
+    take = len(m) if p >= 1 else min(len(m), int(np.searchsorted(cum, p, side="left")) + 1)
+    last = m[order[take - 1]]
+    gap = (last - m[order[take]]) / last if take < len(m) else np.inf
+    tsum = min(abs(cum[take - 1] - p), abs(cum[take - 1] - last - p)) / p if p < 1 else np.inf
+    return np.sort(order[:take]), len(m), gap, tsum
+
+
 def kept_mass(K, q, beta: float, sel, C: int, n1: int) -> float:
     """Share of the dense attention of ``q`` held by the chosen chunks plus tail."""
     K = _f64(K)

@@ -415,3 +415,39 @@ def test_dense_scan_matches_oracle(N, d, dtype, Hq, nq):
                     s, gap, sd = O.dense_scan(Kd, Qh[b, hq, i], beta, mode, p, k)
                     compare_selection(sel, cnt, {wi: _Sel(s, gap, sd)})
     tree.close()
+
+
+@pytest.mark.parametrize("N,d,dtype,Hq,nq,group", [(4096, 64, torch.float32, 1, 8, 16),
+                                                   (3001, 128, torch.bfloat16, 4, 2, 16),
+                                                   (1000, 64, torch.float32, 1, 4, 1),
+                                                   (70001, 128, torch.bfloat16, 4, 1, 16)])
+def test_chunk_mass_matches_oracle(N, d, dtype, Hq, nq, group):
+    """The chunk-mass profile: per walk the fewest chunks of `group` keys holding p
+    of the dense attention, against the oracle (selections may part only at an
+    oracle near-tie); with chunks of one key it is the full-scan indexer."""
+    Z = zha()
+    K, V, refs, Q = _tiny(N, C=8, depth=3, d=d, R=4, B=2, H=1, Hq=Hq, nq=nq, dtype=dtype, seed=N % 89)
+    beta = 1 / np.sqrt(d)
+    tree = Z.Tree(K, V, refs, N, 8, 3, beta)
+    Qh = host64(Q)
+    for p in (0.9, 0.5, 1.0):
+        sel, cnt, n_chunks = tree.chunk_mass(Q, group, p)
+        tree.sync_status()
+        assert n_chunks == (N + group - 1) // group
+        sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+        for b in range(2):
+            Kd = host64(K[b, 0, :N])
+            for hq in range(Hq):
+                for i in range(nq):
+                    wi = (b * Hq + hq) * nq + i
+                    s, nc, gap, sd = O.chunk_mass(Kd, Qh[b, hq, i], beta, group, p)
+                    assert nc == n_chunks
+                    compare_selection(sel, cnt, {wi: _Sel(s, gap, sd)})
+    if group == 1:
+        s1, c1 = tree.dense_scan(Q, O.TOP_P, 0.9, 0)
+        s2, c2, _ = tree.chunk_mass(Q, 1, 0.9)
+        tree.sync_status()
+        assert torch.equal(c1, c2)
+        for w in range(c1.numel()):
+            assert torch.equal(s1[w, : c1[w]], s2[w, : c2[w]])
+    tree.close()

@@ -348,6 +348,44 @@ def test_append_grows_the_depth_at_a_full_top_group():
             assert list(w.sel) == _brute_walk(grown, q, mode, p, k, 2)
 
 
+def test_chunk_mass_of_single_keys_is_the_dense_scan():
+    # chunks of one key: the fewest keys reaching p, the full-scan indexer's top-p
+    # (computed by the C oracle, independently)
+    rng = np.random.default_rng(12)
+    K = rng.standard_normal((500, 16))
+    for i in range(6):
+        q = rng.standard_normal(16) * (0.5 + i)
+        for p in (0.5, 0.9, 0.99):
+            sel, n_chunks, gap, tsum = O.chunk_mass(K, q, 0.7, group=1, p=p)
+            ref, _, _ = O.dense_scan(K, q, 0.7, O.TOP_P, p, 0)
+            assert n_chunks == 500 and list(sel) == list(ref), (i, p)
+
+
+def test_chunk_mass_closed_forms():
+    rng = np.random.default_rng(13)
+    # q = 0: every key weighs 1/n, so a chunk weighs its key count / n.
+    # 64 keys in 4 chunks of 16: 0.25 each, exact in binary: p = 0.75 takes 3, 0.9 takes 4
+    K = rng.standard_normal((64, 8))
+    q = np.zeros(8)
+    sel, n_chunks, _, _ = O.chunk_mass(K, q, 1.0, 16, 0.75)
+    assert n_chunks == 4 and list(sel) == [0, 1, 2]
+    assert list(O.chunk_mass(K, q, 1.0, 16, 0.9)[0]) == [0, 1, 2, 3]
+    assert list(O.chunk_mass(K, q, 1.0, 16, 0.5)[0]) == [0, 1]
+    # 40 keys: chunks of 16, 16 and a partial 8 weigh 0.4, 0.4, 0.2; ties to the lower chunk
+    K = rng.standard_normal((40, 8))
+    sel, n_chunks, _, _ = O.chunk_mass(K, np.zeros(8), 1.0, 16, 0.3)
+    assert n_chunks == 3 and list(sel) == [0]
+    assert list(O.chunk_mass(K, np.zeros(8), 1.0, 16, 0.9)[0]) == [0, 1, 2]
+    # one key far above the rest: its chunk alone holds almost all the mass
+    K = rng.standard_normal((256, 8)) * 0.01
+    K[37] = 10.0
+    q = np.ones(8)
+    sel, n_chunks, _, _ = O.chunk_mass(K, q, 1.0, 16, 0.9)
+    assert n_chunks == 16 and list(sel) == [37 // 16]
+    # p >= 1 takes every chunk
+    assert list(O.chunk_mass(K, q, 1.0, 16, 1.0)[0]) == list(range(16))
+
+
 def test_attend_on_a_subset_is_softmax_attention():
     rng = np.random.default_rng(10)
     N, d, C = 333, 12, 4

@@ -28,7 +28,7 @@ TOP_P, TOP_K = 0, 1
 SYMBOLS = ("zha_build", "zha_append", "zha_search", "zha_attend", "zha_reserve", "zha_level",
            "zha_num_keys", "zha_depth", "zha_sync_status", "zha_destroy", "zha_last_error", "zha_version",
            "zha_profile", "zha_profile_read", "zha_kernel_launches", "zha_last_search_info",
-           "zha_dense_scan", "zha_attend_noalloc")
+           "zha_dense_scan", "zha_attend_noalloc", "zha_chunk_mass")
 KERNEL_KINDS = ("build", "append", "search_init", "score", "select", "attend_plan", "attend_partial",
                 "attend_combine", "score_tc")
 
@@ -81,6 +81,7 @@ def lib():
         L.zha_attend_noalloc.argtypes = [vp, vp, i, i, i, vp, vp, i, vp, i, vp, vp]
         L.zha_reserve.argtypes = [vp, ll, i]
         L.zha_dense_scan.argtypes = [vp, vp, i, i, i, i, f, i, vp, vp, i, vp]
+        L.zha_chunk_mass.argtypes = [vp, vp, i, i, i, i, f, vp, vp, i, vp]
         L.zha_level.argtypes = [vp, i, ctypes.POINTER(vp), ctypes.POINTER(ll), ctypes.POINTER(ll),
                                 ctypes.POINTER(i)]
         L.zha_num_keys.argtypes = [vp]
@@ -263,6 +264,26 @@ class Tree:
         _check(lib().zha_dense_scan(self._h, _dev(Q, "Q"), _dtype_code(Q), Hq, nq, mode, float(p), int(k),
                                     _dev(sel, "sel"), _dev(cnt, "sel_count"), max_sel, _stream(stream)))
         return sel, cnt
+
+    def chunk_mass(self, Q: torch.Tensor, group: int = 16, p: float = 0.9, max_sel: int | None = None, out=None,
+                   stream=None):
+        """Chunk-mass profile of dense attention: per walk, the fewest chunks of
+        `group` keys holding p of the softmax over all keys. Returns (sel
+        [walks][max_sel] int32 chunk indices ascending, count [walks] int32,
+        n_chunks)."""
+        B, Hq, nq, d = Q.shape
+        W = B * Hq * nq
+        n_chunks = (self.n_keys + group - 1) // group if group >= 1 else 0
+        if max_sel is None:
+            max_sel = max(1, n_chunks)
+        if out is None:
+            sel = torch.empty(W, max_sel, dtype=torch.int32, device=Q.device)
+            cnt = torch.empty(W, dtype=torch.int32, device=Q.device)
+        else:
+            sel, cnt = out
+        _check(lib().zha_chunk_mass(self._h, _dev(Q, "Q"), _dtype_code(Q), Hq, nq, int(group), float(p),
+                                    _dev(sel, "sel"), _dev(cnt, "count"), max_sel, _stream(stream)))
+        return sel, cnt, n_chunks
 
     def reserve(self, max_walks: int, max_sel: int) -> None:
         _check(lib().zha_reserve(self._h, int(max_walks), int(max_sel)))

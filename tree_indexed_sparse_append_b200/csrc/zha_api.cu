@@ -388,6 +388,47 @@ int zha_attend(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads, int
     return ZHA_OK;
 }
 
+// Grows the tree's full-scan scratch to at least `need` bytes.
+static int grow_dense_scratch(zha_tree *t, size_t need) {
+    if (need <= t->dws_bytes) return ZHA_OK;
+    if (t->dws) cudaFree(t->dws);
+    t->dws = nullptr;
+    t->dws_bytes = 0;
+    cudaError_t e = cudaMalloc(&t->dws, need);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_fail(e, "allocating full-scan scratch");
+    }
+    t->dws_bytes = need;
+    return ZHA_OK;
+}
+
+int zha_chunk_mass(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q, int group, float p,
+                   int *sel, int *count, int max_sel, void *stream) {
+    long long W;
+    int G;
+    int rc = check_queries(t, Q, q_dtype, n_q_heads, n_q, &W, &G);
+    if (rc) return rc;
+    if (G > 32) return fail(ZHA_ERR_INVALID, "the chunk-mass profile takes at most 32 walks per tree (got %d)", G);
+    if (group < 1) return fail(ZHA_ERR_INVALID, "group must be >= 1 (got %d)", group);
+    if (!(p > 0.f) || std::isnan(p)) return fail(ZHA_ERR_INVALID, "p must be > 0 (got %g)", (double)p);
+    if (!sel || !count) return fail(ZHA_ERR_INVALID, "sel and count must not be NULL");
+    if (max_sel < 1) return fail(ZHA_ERR_INVALID, "max_sel must be >= 1");
+    const long long N = t->n > 0 ? t->n : 1;
+    const long long nch = (N + group - 1) / group;
+    const size_t o_S = align_up(sizeof(float) * W * t->cfg.d);
+    const size_t o_Sc = o_S + align_up(sizeof(float) * W * N);
+    const size_t o_gk = o_Sc + align_up(sizeof(float) * W * nch);
+    rc = grow_dense_scratch(t, o_gk + align_up(sizeof(uint32_t) * W * nch));
+    if (rc) return rc;
+    char *b = static_cast<char *>(t->dws);
+    ZHA_CUDA(zha::launch_chunk_mass(t, Q, q_dtype, G, W, group, p, sel, count, max_sel, reinterpret_cast<float *>(b),
+                                    reinterpret_cast<float *>(b + o_S), reinterpret_cast<float *>(b + o_Sc),
+                                    reinterpret_cast<uint32_t *>(b + o_gk), static_cast<cudaStream_t>(stream)),
+             "launching the chunk-mass profile");
+    return ZHA_OK;
+}
+
 int zha_dense_scan(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q, zha_mode mode, float p,
                    int k, int *sel, int *sel_count, int max_sel, void *stream) {
     long long W;
@@ -407,17 +448,8 @@ int zha_dense_scan(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads,
     const long long N = t->n > 0 ? t->n : 1;
     const size_t need = align_up(sizeof(float) * W * t->cfg.d) + align_up(sizeof(float) * W * N) +
                         align_up(sizeof(uint32_t) * W * N);
-    if (need > t->dws_bytes) {
-        if (t->dws) cudaFree(t->dws);
-        t->dws = nullptr;
-        t->dws_bytes = 0;
-        cudaError_t e = cudaMalloc(&t->dws, need);
-        if (e != cudaSuccess) {
-            cudaGetLastError();
-            return cuda_fail(e, "allocating full-scan scratch");
-        }
-        t->dws_bytes = need;
-    }
+    rc = grow_dense_scratch(t, need);
+    if (rc) return rc;
     char *b = static_cast<char *>(t->dws);
     float *qf = reinterpret_cast<float *>(b);
     float *S = reinterpret_cast<float *>(b + align_up(sizeof(float) * W * t->cfg.d));

@@ -15,6 +15,12 @@
 //              U * GP = 32), and one warp transpose-reduce leaves every lane
 //              with one (key, walk) score.
 // select       the tree walk's selector with every key in the frontier.
+//
+// Chunk-mass profile (same page set, "How does top-p differ from top-K?": how
+// many 16-key chunks hold 90% of a query's attention varies a lot by task): the
+// dense scores above, reduced per run of `group` keys to the chunk's
+// log-sum-exp, so that the softmax over chunk scores is the chunk's share of the
+// dense attention; the selector then opens the fewest chunks reaching p.
 #include <algorithm>
 
 #include "zha_internal.cuh"
@@ -137,11 +143,28 @@ cudaError_t dense_score_g(const zha_tree *t, const DenseArgs &a, cudaStream_t st
     return launch_dense_score<T, D, 32>(t, a, st);
 }
 
-}  // namespace
+// S[w][c] of the chunk-mass profile: log sum_j exp(s_j) over the keys
+// c*group .. min(c*group + group, N) - 1 of the walk's dense scores (fp32).
+__global__ void chunk_lse_kernel(const float *S, long long N, int group, long long nch, long long W, float *Sc) {
+    chain_start();
+    const long long total = W * nch;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const long long w = i / nch, c = i - w * nch;
+        const float *row = S + w * N + c * group;
+        const int cnt = (int)(N - c * group < group ? N - c * group : group);
+        float m = -INFINITY;
+        for (int j = 0; j < cnt; ++j) m = fmaxf(m, row[j]);
+        float sum = 0.f;
+        for (int j = 0; j < cnt; ++j) sum += expf(row[j] - m);
+        Sc[i] = m + logf(sum);
+    }
+    chain_done();
+}
 
-cudaError_t launch_dense_scan(const zha_tree *t, const void *Q, zha_dtype q_dtype, int G, long long W, int mode,
-                              float p, int k, int *sel, int *sel_count, int max_sel, float *qf, float *S,
-                              uint32_t *gkey, cudaStream_t st) {
+// Queries to fp32, then every key's score for every walk of its tree into S.
+cudaError_t dense_scores(const zha_tree *t, const void *Q, zha_dtype q_dtype, int G, long long W, float *qf,
+                         float *S, cudaStream_t st) {
     const zha_config &c = t->cfg;
     const long long nq = W * c.d;
     {
@@ -160,17 +183,42 @@ cudaError_t launch_dense_scan(const zha_tree *t, const void *Q, zha_dtype q_dtyp
     a.beta = c.sharpness;
     a.qf = qf;
     a.S = S;
-    cudaError_t e = cudaSuccess;
-    if (a.N > 0) {
-        const bool bf = c.kv_dtype == ZHA_BF16;
-        switch (c.d) {
-            case 64: e = bf ? dense_score_g<__nv_bfloat16, 64>(t, a, st) : dense_score_g<float, 64>(t, a, st); break;
-            case 128: e = bf ? dense_score_g<__nv_bfloat16, 128>(t, a, st) : dense_score_g<float, 128>(t, a, st); break;
-            default: e = bf ? dense_score_g<__nv_bfloat16, 256>(t, a, st) : dense_score_g<float, 256>(t, a, st); break;
-        }
+    if (a.N <= 0) return cudaSuccess;
+    const bool bf = c.kv_dtype == ZHA_BF16;
+    switch (c.d) {
+        case 64: return bf ? dense_score_g<__nv_bfloat16, 64>(t, a, st) : dense_score_g<float, 64>(t, a, st);
+        case 128: return bf ? dense_score_g<__nv_bfloat16, 128>(t, a, st) : dense_score_g<float, 128>(t, a, st);
+        default: return bf ? dense_score_g<__nv_bfloat16, 256>(t, a, st) : dense_score_g<float, 256>(t, a, st);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_mass(const zha_tree *t, const void *Q, zha_dtype q_dtype, int G, long long W, int group,
+                              float p, int *sel, int *count, int max_sel, float *qf, float *S, float *Sc,
+                              uint32_t *gkey, cudaStream_t st) {
+    cudaError_t e = dense_scores(t, Q, q_dtype, G, W, qf, S, st);
+    if (e != cudaSuccess) return e;
+    const long long N = t->n;
+    const long long nch = (N + group - 1) / group;
+    if (nch > 0) {
+        Probe pr(t, ZHA_K_SCORE, st);
+        const long long total = W * nch;
+        const long long blocks = std::min<long long>((total + 255) / 256, 8LL * num_sms());
+        launch_chained(chunk_lse_kernel, dim3((unsigned)blocks), dim3(256), 0, st, (const float *)S, N, group,
+                       nch, W, Sc);
+        e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    return launch_select_all(t, S, gkey, a.N, W, G, mode, p, k, sel, sel_count, max_sel, st);
+    return launch_select_all(t, Sc, gkey, nch, W, G, ZHA_TOP_P, p, 0, sel, count, max_sel, st);
+}
+
+cudaError_t launch_dense_scan(const zha_tree *t, const void *Q, zha_dtype q_dtype, int G, long long W, int mode,
+                              float p, int k, int *sel, int *sel_count, int max_sel, float *qf, float *S,
+                              uint32_t *gkey, cudaStream_t st) {
+    cudaError_t e = dense_scores(t, Q, q_dtype, G, W, qf, S, st);
+    if (e != cudaSuccess) return e;
+    return launch_select_all(t, S, gkey, t->n, W, G, mode, p, k, sel, sel_count, max_sel, st);
 }
 
 }  // namespace zha

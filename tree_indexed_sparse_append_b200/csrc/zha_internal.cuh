@@ -284,6 +284,11 @@ cudaError_t launch_select_all(const zha_tree *t, const float *S, uint32_t *gkey,
 cudaError_t launch_dense_scan(const zha_tree *t, const void *Q, zha_dtype q_dtype, int G, long long W, int mode,
                               float p, int k, int *sel, int *sel_count, int max_sel, float *qf, float *S,
                               uint32_t *gkey, cudaStream_t st);
+// Chunk-mass profile: dense scores into S [W][N], chunk log-sum-exps into
+// Sc [W][ceil(N / group)], then top-p over each walk's chunks.
+cudaError_t launch_chunk_mass(const zha_tree *t, const void *Q, zha_dtype q_dtype, int G, long long W, int group,
+                              float p, int *sel, int *count, int max_sel, float *qf, float *S, float *Sc,
+                              uint32_t *gkey, cudaStream_t st);
 
 int num_sms();
 
