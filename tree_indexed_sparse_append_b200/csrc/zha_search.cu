@@ -947,6 +947,11 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
                 // many walks (prefill): 512 threads keep two CTAs per SM
                 se.smem_keys = std::min<long long>(t->n_nodes[l], 16384);
                 e = W <= 2LL * num_sms() ? launch_select<1024>(se, W, st) : launch_select<512>(se, W, st);
+            } else if (t->n_nodes[l] > 2048 && W <= 2LL * num_sms()) {
+                // few walks over a level of thousands of nodes: frontiers of a few
+                // thousand keys, 512 threads
+                se.smem_keys = t->n_nodes[l];
+                e = launch_select<512>(se, W, st);
             } else {
                 se.smem_keys = t->n_nodes[l];
                 e = launch_select<256>(se, W, st);
