@@ -23,11 +23,14 @@
 //                scored against every walk whose frontier holds it (a ballot over
 //                per-walk membership bits). Dot products reduce with a warp
 //                transpose-reduce (R rows in R-1+5-log2 R shuffles).
-//   select_level One CTA per walk. Exact selection without sorting: a 4-pass
-//                8-bit radix select over the fp32 score bits, where each bucket
-//                carries its count and its softmax mass in 40-bit fixed point
-//                (integer sums: exact and order-independent). Ties at the
-//                boundary score open in ascending node id. Opened nodes are
+//   select_level One CTA per walk. Exact selection without sorting: histogram
+//                passes over 256 buckets (1/8-nat buckets below the frontier's
+//                maximum, then 1/2048-nat buckets inside the crossing one, then
+//                the raw score bytes), each bucket carrying its count and its
+//                softmax mass in 40-bit fixed point (integer sums: exact and
+//                order-independent); a crossing bucket of at most 32 keys is
+//                ranked directly by one warp. Ties at the boundary score open
+//                in ascending node id. Opened nodes are
 //                compacted in id order by block scans; their children and the
 //                orphans of the level below form the next frontier (membership
 //                bits per walk and a per-tree union).
