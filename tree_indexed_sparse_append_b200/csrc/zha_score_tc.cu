@@ -31,6 +31,15 @@
 //                    (2 tiles x 2 buffers = all 512 TMEM columns); eight epilogue
 //                    warps read a finished accumulator back (tcgen05.ld), free it,
 //                    take the max over references and store the scores.
+//   Levels of more than 8,192 nodes are not computed whole (the walks' frontiers
+//   cover a small part of them):
+//   tc_members       per tree and tile of 16 nodes (one word of the membership
+//                    bitmap), the list of walks whose frontier holds one of them.
+//   score_tc_sparse_kernel  one CTA per tile with members: the tile's three key
+//                    parts and biases in shared memory (one bulk copy), the member
+//                    walks' queries gathered 128 at a time (cp.async, zero-filled
+//                    past the end), the same MMAs into 128 TMEM columns, and scores
+//                    stored for the member walks only.
 // Every wait is bounded: on timeout the kernel records DEV_TIMEOUT, waits (also
 // bounded) for its own copies and MMAs, frees its TMEM and returns.
 #include <cstdint>
