@@ -11,7 +11,10 @@ Workload (N=1 headline): 16 sequences x 4 KV heads x 262,144 keys, 16 query head
 0.9, one query per head: 256 walks per step; clustered synthetic keys (blocks of
 64 around N(0, I) centres, noise 0.3), queries mixing 1-8 centres. Also reported:
 the 1,048,576-key workload (8 x 8 KV heads, 32 query heads, chunk 16, 5 levels,
-top-p 0.9 and top-K 16).
+top-p 0.9 and top-K 16) with the full-scan indexer and the chunk-mass profile of
+dense attention on the same trees, and the prefill workload (4,096 queries x 16
+query heads against one sequence's four 262,144-key trees, scored on the tensor
+cores).
 
 Under torchrun each rank runs its own copy of the workload (distinct seeds) on its
 GPU: weak scaling, no data-path collective; time = max over ranks.
