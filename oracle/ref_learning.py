@@ -92,3 +92,89 @@ def learn_refs(K: torch.Tensor, refs0: torch.Tensor, Q: torch.Tensor, C: int, de
             refs -= lr * g
     losses.append(float(split_loss(K, refs.detach(), Q, C, depth, beta)))
     return refs.detach(), losses
+
+
+def _lse(x, axis: int):
+    import numpy as np
+
+    m = x.max(axis=axis, keepdims=True)
+    return np.log(np.exp(x - m).sum(axis=axis)) + np.squeeze(m, axis=axis)
+
+
+def split_loss_and_grad(K, refs, Q, C: int, depth: int, beta: float):
+    """The split loss and its gradient with respect to the references, written out
+    (numpy, double precision, no autograd): the backward pass a GPU version
+    follows. Per level l and query m, with g = (tree split - teacher split) / m_q
+    on the node scores:
+      - a node score is beta*<key_{j,r*}, q> + bias_{j,r*} at its best reference
+        r*, so g flows to key_{j,r*} as g*beta*q and to bias_{j,r*} as g;
+      - a node (j, r) built from children i with s_i = beta*<c_i, q_r> + b_i,
+        w = softmax(s), key = sum_i w_i c_i, bias = logsumexp(s) - beta*<key, q_r>
+        passes on, with Gk = G_key - beta*G_bias*q_r and
+        G_s_i = w_i*(<Gk, c_i> - <Gk, key> + G_bias):
+          to its children: G_c_i += w_i*Gk + beta*G_s_i*q_r, G_b_i += G_s_i;
+          to its reference: G_q_r += beta*(sum_i G_s_i*c_i - G_bias*key);
+    taken from the top level down, each level's node gradients being its own loss
+    term's plus what its parents pass on. Returns (loss, gradient [R][d])."""
+    import numpy as np
+
+    K = np.asarray(K, dtype=np.float64)
+    refs = np.asarray(refs, dtype=np.float64)
+    Q = np.asarray(Q, dtype=np.float64)
+    R, d = refs.shape
+    m_q = Q.shape[0]
+    # forward, keeping every level's children
+    levels = []  # (child keys [R][n][C][d], child biases [R][n][C], w [R][n][C], key [R][n][d])
+    ck_all = np.broadcast_to(K[None], (R,) + K.shape)
+    cb_all = np.zeros((R, K.shape[0]))
+    for _ in range(depth):
+        n = ck_all.shape[1] // C
+        ck = ck_all[:, : n * C].reshape(R, n, C, d)
+        cb = cb_all[:, : n * C].reshape(R, n, C)
+        s = beta * np.einsum("rncd,rd->rnc", ck, refs) + cb
+        lse = _lse(s, 2) if n else np.zeros((R, 0))
+        w = np.exp(s - lse[..., None])
+        key = np.einsum("rnc,rncd->rnd", w, ck)
+        bias = lse - beta * np.einsum("rnd,rd->rn", key, refs)
+        levels.append((ck, cb, w, key, bias))
+        ck_all, cb_all = key, bias
+    # loss terms and the score gradients of every level
+    logits = beta * Q @ K.T
+    loss = 0.0
+    G_key = [np.zeros_like(lv[3]) for lv in levels]   # [R][n][d] per level
+    G_bias = [np.zeros_like(lv[4]) for lv in levels]  # [R][n]
+    for li, (ck, cb, w, key, bias) in enumerate(levels):
+        n = key.shape[1]
+        if n == 0:
+            continue
+        span = C ** (li + 1)
+        blocks = logits[:, : n * span].reshape(m_q, n, span)
+        logP = _lse(blocks, 2)                    # log dense mass under each node
+        logP = logP - _lse(logP, 1)[:, None]      # over the keys the level covers
+        per_r = beta * np.einsum("rnd,md->mnr", key, Q) + bias.T[None]  # [m][n][R]
+        best = per_r.argmax(axis=2)
+        score = np.take_along_axis(per_r, best[..., None], axis=2)[..., 0]
+        logT = score - _lse(score, 1)[:, None]
+        P = np.exp(logP)
+        loss += float((P * (logP - logT)).sum(axis=1).mean())
+        g = (np.exp(logT) - P) / m_q  # [m][n]
+        for r in range(R):
+            sel = (best == r) * g  # [m][n]
+            G_key[li][r] += beta * sel.T @ Q
+            G_bias[li][r] += sel.sum(axis=0)
+    # backward through the build, top level first
+    grad = np.zeros_like(refs)
+    for li in range(len(levels) - 1, -1, -1):
+        ck, cb, w, key, bias = levels[li]
+        if key.shape[1] == 0:
+            continue
+        Gb = G_bias[li]                                          # [R][n]
+        Gk = G_key[li] - beta * Gb[..., None] * refs[:, None, :]  # [R][n][d]
+        Gs = w * (np.einsum("rnd,rncd->rnc", Gk, ck) - np.einsum("rnd,rnd->rn", Gk, key)[..., None] + Gb[..., None])
+        grad += beta * (np.einsum("rnc,rncd->rd", Gs, ck) - np.einsum("rn,rnd->rd", Gb, key))
+        if li > 0:
+            n = key.shape[1]
+            Gc = w[..., None] * Gk[:, :, None, :] + beta * Gs[..., None] * refs[:, None, None, :]
+            G_key[li - 1][:, : n * C] += Gc.reshape(R, n * C, d)
+            G_bias[li - 1][:, : n * C] += Gs.reshape(R, n * C)
+    return loss, grad

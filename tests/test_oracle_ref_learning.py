@@ -87,3 +87,17 @@ def test_descent_lowers_the_loss():
     refs, losses = RL.learn_refs(K, refs0, Q, C, depth, beta, steps=60, lr=0.5)
     assert losses[-1] < 0.7 * losses[0], losses[::10]
     assert all(np.isfinite(losses))
+
+
+@pytest.mark.parametrize("N,C,depth,R", [(256, 4, 4, 3), (300, 4, 3, 2), (200, 3, 4, 4)])
+def test_written_out_gradient_equals_autograd(N, C, depth, R):
+    # the explicit backward (the one a GPU version follows) against torch's autograd
+    d, beta = 8, 0.6
+    K, centres, g = _keys(N, d, 10 + N)
+    Q = centres[torch.randint(0, len(centres), (5,), generator=g)] * 1.5 + 0.1 * _randn(5, d, g=g)
+    refs = _randn(R, d, g=g).requires_grad_(True)
+    loss = RL.split_loss(K, refs, Q, C, depth, beta)
+    (ga,) = torch.autograd.grad(loss, refs)
+    l2, g2 = RL.split_loss_and_grad(K.numpy(), refs.detach().numpy(), Q.numpy(), C, depth, beta)
+    assert abs(l2 - loss.item()) <= 1e-12 * max(1.0, abs(loss.item()))
+    np.testing.assert_allclose(g2, ga.numpy(), rtol=0, atol=1e-12 * max(1.0, np.abs(ga.numpy()).max()))
