@@ -232,6 +232,25 @@ int zha_chunk_mass(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_hea
                    int *sel, int *count, int max_sel, void *stream);
 
 /*
+ * zha_ref_grad: the loss that teaches the reference queries, and its gradient
+ * ([P1] "Does the model have to be retrained?": the model stays frozen and the
+ * reference queries are learned by comparing how the tree splits attention with
+ * how the model does, by KL distillation). At every level l the tree splits a
+ * query's attention as softmax_j(max_r(beta*<key_{j,r}, q> + bias_{j,r})); the
+ * teacher splits it as the dense attention mass under each node, over the
+ * C^l * n_l keys the level covers. loss = mean over the walks of the sum over
+ * levels of KL(teacher || tree); grad = d loss / d refs, for the refs the tree
+ * was built with (rebuild with zha_build after updating them).
+ * Q:    [B][H_q][n_q][d] of q_dtype; at most 32 walks per tree.
+ * loss: device float[1]; grad: device float [H_kv][R][d] (both overwritten).
+ * Scratch of about 4 * walks * (n + 4 * n_1) + 4 * trees * R * (d + 1) * (sum of
+ * the level sizes) bytes is allocated on `stream` and freed there.
+ * Errors: ZHA_ERR_INVALID, ZHA_ERR_OOM, ZHA_ERR_CUDA.
+ */
+int zha_ref_grad(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q, float *loss, float *grad,
+                 void *stream);
+
+/*
  * zha_reserve: allocate the search and attend scratch for up to max_walks walks
  * and selections of up to max_sel chunks now, so that later calls with at most
  * these sizes allocate nothing (e.g. before capturing them in a CUDA graph).

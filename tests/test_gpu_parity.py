@@ -451,3 +451,33 @@ def test_chunk_mass_matches_oracle(N, d, dtype, Hq, nq, group):
         for w in range(c1.numel()):
             assert torch.equal(s1[w, : c1[w]], s2[w, : c2[w]])
     tree.close()
+
+
+@pytest.mark.parametrize("dtype,d,C,depth", [(torch.float32, 64, 4, 4), (torch.bfloat16, 128, 8, 3)])
+def test_ref_grad_matches_oracle(dtype, d, C, depth):
+    """The split loss and its gradient with respect to the references against the
+    CPU reference (explicit backward in double precision)."""
+    from oracle import ref_learning as RL
+
+    Z = zha()
+    B, H, R, Hq, nq = 1, 2, 3, 4, 2
+    N = C ** depth * 2 + 37  # a tail past the last full node
+    K, V, refs, Q = _tiny(N, C=C, d=d, R=R, B=B, H=H, Hq=Hq, nq=nq, dtype=dtype, seed=9)
+    beta = 0.3
+    tree = Z.Tree(K, V, refs, N, C, depth, beta)
+    loss, grad = tree.ref_grad(Q)
+    tree.sync_status()
+    loss, grad = float(loss.item()), grad.double().cpu().numpy()
+    group = Hq // H
+    Qh = host64(Q)
+    losses, grads = [], []
+    for h in range(H):
+        q = Qh[0, h * group: (h + 1) * group].reshape(-1, d)
+        lo, go = RL.split_loss_and_grad(host64(K[0, h, :N]), host64(refs[h]), q, C, depth, beta)
+        losses.append(lo)
+        grads.append(go / H)  # the GPU averages over all walks of all trees
+    assert abs(loss - np.mean(losses)) <= 2e-4 * max(1.0, abs(np.mean(losses))), (loss, losses)
+    for h in range(H):
+        scale = max(1e-6, np.abs(grads[h]).max())
+        assert np.abs(grad[h] - grads[h]).max() <= 2e-3 * scale, (h, np.abs(grad[h] - grads[h]).max(), scale)
+    tree.close()

@@ -28,7 +28,7 @@ TOP_P, TOP_K = 0, 1
 SYMBOLS = ("zha_build", "zha_append", "zha_search", "zha_attend", "zha_reserve", "zha_level",
            "zha_num_keys", "zha_depth", "zha_sync_status", "zha_destroy", "zha_last_error", "zha_version",
            "zha_profile", "zha_profile_read", "zha_kernel_launches", "zha_last_search_info",
-           "zha_dense_scan", "zha_attend_noalloc", "zha_chunk_mass")
+           "zha_dense_scan", "zha_attend_noalloc", "zha_chunk_mass", "zha_ref_grad")
 KERNEL_KINDS = ("build", "append", "search_init", "score", "select", "attend_plan", "attend_partial",
                 "attend_combine", "score_tc")
 
@@ -82,6 +82,7 @@ def lib():
         L.zha_reserve.argtypes = [vp, ll, i]
         L.zha_dense_scan.argtypes = [vp, vp, i, i, i, i, f, i, vp, vp, i, vp]
         L.zha_chunk_mass.argtypes = [vp, vp, i, i, i, i, f, vp, vp, i, vp]
+        L.zha_ref_grad.argtypes = [vp, vp, i, i, i, vp, vp, vp]
         L.zha_level.argtypes = [vp, i, ctypes.POINTER(vp), ctypes.POINTER(ll), ctypes.POINTER(ll),
                                 ctypes.POINTER(i)]
         L.zha_num_keys.argtypes = [vp]
@@ -284,6 +285,18 @@ class Tree:
         _check(lib().zha_chunk_mass(self._h, _dev(Q, "Q"), _dtype_code(Q), Hq, nq, int(group), float(p),
                                     _dev(sel, "sel"), _dev(cnt, "count"), max_sel, _stream(stream)))
         return sel, cnt, n_chunks
+
+    def ref_grad(self, Q: torch.Tensor, stream=None):
+        """The split loss (KL of the teacher's split of attention from the tree's,
+        summed over levels, averaged over walks) and its gradient with respect to
+        the references the tree was built with. Returns (loss [1], grad
+        [H_kv][R][d]), fp32 on the device."""
+        B, Hq, nq, d = Q.shape
+        loss = torch.empty(1, dtype=torch.float32, device=Q.device)
+        grad = torch.empty(self.cfg.n_kv_heads, self.cfg.R, d, dtype=torch.float32, device=Q.device)
+        _check(lib().zha_ref_grad(self._h, _dev(Q, "Q"), _dtype_code(Q), Hq, nq, _dev(loss, "loss"),
+                                  _dev(grad, "grad"), _stream(stream)))
+        return loss, grad
 
     def reserve(self, max_walks: int, max_sel: int) -> None:
         _check(lib().zha_reserve(self._h, int(max_walks), int(max_sel)))

@@ -194,6 +194,21 @@ cudaError_t dense_scores(const zha_tree *t, const void *Q, zha_dtype q_dtype, in
 
 }  // namespace
 
+cudaError_t launch_dense_scores(const zha_tree *t, const void *Q, zha_dtype q_dtype, int G, long long W, float *qf,
+                                float *S, cudaStream_t st) {
+    return dense_scores(t, Q, q_dtype, G, W, qf, S, st);
+}
+
+cudaError_t launch_chunk_lse(const zha_tree *t, const float *S, long long N, int group, long long nch, long long W,
+                             float *Sc, cudaStream_t st) {
+    if (nch <= 0 || W <= 0) return cudaSuccess;
+    Probe pr(t, ZHA_K_SCORE, st);
+    const long long total = W * nch;
+    const long long blocks = std::min<long long>((total + 255) / 256, 8LL * num_sms());
+    launch_chained(chunk_lse_kernel, dim3((unsigned)blocks), dim3(256), 0, st, S, N, group, nch, W, Sc);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_chunk_mass(const zha_tree *t, const void *Q, zha_dtype q_dtype, int G, long long W, int group,
                               float p, int *sel, int *count, int max_sel, float *qf, float *S, float *Sc,
                               uint32_t *gkey, cudaStream_t st) {

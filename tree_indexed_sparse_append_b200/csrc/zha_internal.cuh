@@ -284,6 +284,13 @@ cudaError_t launch_select_all(const zha_tree *t, const float *S, uint32_t *gkey,
 cudaError_t launch_dense_scan(const zha_tree *t, const void *Q, zha_dtype q_dtype, int G, long long W, int mode,
                               float p, int k, int *sel, int *sel_count, int max_sel, float *qf, float *S,
                               uint32_t *gkey, cudaStream_t st);
+// Queries to fp32 (qf [W][d]) and every key's score beta*<q, k> into S [W][n]
+// (at most 32 walks per tree).
+cudaError_t launch_dense_scores(const zha_tree *t, const void *Q, zha_dtype q_dtype, int G, long long W, float *qf,
+                                float *S, cudaStream_t st);
+// Sc[w][c] = log sum_j exp(S[w][c*group + j]) over the chunk's keys (rows of N).
+cudaError_t launch_chunk_lse(const zha_tree *t, const float *S, long long N, int group, long long nch, long long W,
+                             float *Sc, cudaStream_t st);
 // Chunk-mass profile: dense scores into S [W][N], chunk log-sum-exps into
 // Sc [W][ceil(N / group)], then top-p over each walk's chunks.
 cudaError_t launch_chunk_mass(const zha_tree *t, const void *Q, zha_dtype q_dtype, int G, long long W, int group,
