@@ -44,7 +44,6 @@ __global__ void __launch_bounds__(256) node_scores_kernel(const float *nodes, lo
     const int lane = threadIdx.x & 31;
     const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
-    const long long W = (long long)T * G;
     for (long long it = gw; it < (long long)T * n_l; it += nw) {
         const long long t = it / n_l, j = it - t * n_l;
         const float *node = nodes + (t * cap_l + j) * NF;
@@ -72,7 +71,6 @@ __global__ void __launch_bounds__(256) node_scores_kernel(const float *nodes, lo
             }
         }
     }
-    (void)W;
 }
 
 __device__ __forceinline__ float block_reduce(float v, float *sh, bool is_max) {
