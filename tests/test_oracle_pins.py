@@ -386,6 +386,27 @@ def test_chunk_mass_closed_forms():
     assert list(O.chunk_mass(K, q, 1.0, 16, 1.0)[0]) == list(range(16))
 
 
+@pytest.mark.parametrize("seed", range(8))
+def test_chunk_mass_count_is_the_minimum(seed):
+    # no smaller set of chunks reaches p (exhaustive over tiny inputs, exact sums)
+    rng = np.random.default_rng(100 + seed)
+    n, g = int(rng.integers(20, 80)), int(rng.integers(4, 9))
+    K = rng.standard_normal((n, 6))
+    q = rng.standard_normal(6) * rng.uniform(0.5, 3.0)
+    for p in (0.5, 0.8, 0.9):
+        sel, n_chunks, gap, tsum = O.chunk_mass(K, q, 1.0, g, p)
+        if min(gap, tsum) < 1e-12:
+            continue
+        s = K @ q
+        w = np.exp(s - s.max())
+        m = [Fraction(float(x)) for x in np.add.reduceat(w, np.arange(0, n, g))]
+        total = sum(m)
+        assert sum(m[c] for c in sel) >= Fraction(p) * total
+        smaller = [c for c in itertools.combinations(range(n_chunks), len(sel) - 1)
+                   if sum(m[i] for i in c) >= Fraction(p) * total]
+        assert not smaller, (seed, p, len(sel))
+
+
 def test_attend_on_a_subset_is_softmax_attention():
     rng = np.random.default_rng(10)
     N, d, C = 333, 12, 4
