@@ -15,6 +15,11 @@ grows its depth with the keys (page "Subquadratic Attention with a Hierarchical
 Tree-Structured Indexer", abstract: the tree's depth grows with the context): it
 keeps every level that holds a node, and the parent made when a group of C top
 nodes fills starts a new level.
+
+Two modules sit beside it: ``ref_learning.py`` (the loss that teaches the
+reference queries and its gradient, in double precision) and
+``context_parallel.py`` (the walk of one tree whose keys are split across the
+ranks of a process group).
 """
 from __future__ import annotations
 
