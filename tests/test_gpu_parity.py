@@ -5,10 +5,13 @@ tails, orphans, GQA groups, several queries per head).
 What is compared, per workload and mode:
   * every node key and bias of every level of every tree (1e-5 relative);
   * every walk's selected chunk set (identical except at oracle near-ties, which
-    are counted and printed) and its counters (frontier and opened per level,
-    keys read, comparisons);
+    are counted and printed; such a walk must be an admissible walk under the
+    oracle's masses, and at most 1% of the walks, at least one, may part) and its
+    counters (frontier and opened per level, keys read, comparisons);
   * the attention over the oracle's own selection (GPU attend fed the oracle's
-    chunk lists), and the end-to-end search + attend where the sets agree;
+    chunk lists), and the end-to-end search + attend against the oracle's
+    attention over the GPU's selection (the same as the oracle's own, except for
+    a walk that parts at a near-tie);
   * p = 1 against dense attention.
 """
 import numpy as np
@@ -17,8 +20,9 @@ import torch
 
 import oracle as O
 import synthetic as S
-from helpers import (assert_attention_close, assert_bf16_output_close, assert_nodes_close, attn_tol,
-                     compare_selection, gpu_level, host64, oracle_tree)
+from helpers import (assert_attention_close, assert_bf16_output_close, assert_nodes_close,
+                     assert_partings_bounded, attn_tol, compare_selection, gpu_level, host64, one_level_valid,
+                     oracle_tree, tree_walk_valid)
 
 pytestmark = pytest.mark.gpu
 
@@ -69,6 +73,15 @@ class Case:
         return {wi: O.search(self.otrees[key], q, MODE[mode], p, k, self.w.top_width)
                 for wi, key, q in self.walks()}
 
+    def valid(self, mode, p, k):
+        """compare_selection's check that a parting walk is admissible."""
+        where = {wi: (key, q) for wi, key, q in self.walks()}
+
+        def check(wi, g):
+            key, q = where[wi]
+            return tree_walk_valid(self.otrees[key], q, MODE[mode], p, k, self.w.top_width)(wi, g)
+        return check
+
 
 @pytest.fixture(scope="module", params=list(SMALL))
 def case(request):
@@ -102,8 +115,9 @@ def test_search_matches_oracle(case, mode_i):
     sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
     stats = Z.parse_stats(st)
     ow = case.oracle_search(mode, p, k)
-    differ = compare_selection(sel, cnt, ow)
+    differ = compare_selection(sel, cnt, ow, case.valid(mode, p, k))
     print(f"{case.name} {mode}: {len(differ)} of {len(ow)} walks part at oracle near-ties")
+    assert_partings_bounded(len(differ), len(ow), f"{case.name} {mode}")
     for wi, o in ow.items():
         if wi in differ:
             continue
@@ -147,14 +161,16 @@ def test_search_then_attend_end_to_end(case):
     out, lse = case.tree.attend(case.inp.Q, sel, cnt, out_dtype=torch.float32)
     case.tree.sync_status()
     ow = case.oracle_search(mode, p, k)
-    differ = compare_selection(sel.cpu().numpy(), cnt.cpu().numpy(), ow)
+    sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+    differ = compare_selection(sel, cnt, ow, case.valid(mode, p, k))
+    assert_partings_bounded(len(differ), len(ow), f"{case.name} {mode}")
     out = host64(out).reshape(w.walks, w.d)
     lse = lse.cpu().numpy()
     n1 = case.otrees[(0, 0)].n_nodes[1]
     for wi, key, q in case.walks():
-        if wi in differ:
-            continue
-        o_out, o_lse = O.attend(case.Kh[key], case.Vh[key], q, ow[wi].sel, w.chunk, n1, w.beta)
+        # the oracle's attention over the GPU's own selection (the oracle's, unless
+        # the walk parted at a near-tie)
+        o_out, o_lse = O.attend(case.Kh[key], case.Vh[key], q, sel[wi, : cnt[wi]], w.chunk, n1, w.beta)
         assert_attention_close(out[wi], lse[wi], o_out, o_lse, attn_tol(w), f"{case.name} walk {wi}")
 
 
@@ -213,6 +229,7 @@ def _check_against_oracle(K, V, refs, Q, N, C, depth, beta, top_width=64, modes=
                 if n:
                     keys, bias = ot.level(l)
                     assert_nodes_close(g, keys, bias, R, d)
+    parted = walks = 0
     for mode, p, k in modes:
         sel, cnt, st = tree.search(Q, mode, p, k, max_sel=max(1, N // C), with_stats=True)
         out, lse = tree.attend(Q, sel, cnt, out_dtype=torch.float32)
@@ -231,18 +248,22 @@ def _check_against_oracle(K, V, refs, Q, N, C, depth, beta, top_width=64, modes=
                 for i in range(nq):
                     wi = (b * Hq + hq) * nq + i
                     ow = O.search(ot, Qh[b, hq, i], mode, p, k, top_width)
-                    compare_selection(sel, cnt, {wi: ow})
-                    if not np.array_equal(sel[wi, : cnt[wi]], ow.sel):
-                        continue
-                    assert stats[wi]["keys_read"] == ow.keys_read and stats[wi]["work"] == ow.work
+                    parted += len(compare_selection(sel, cnt, {wi: ow},
+                                                    tree_walk_valid(ot, Qh[b, hq, i], mode, p, k, top_width)))
+                    walks += 1
+                    g = sel[wi, : cnt[wi]]
+                    if np.array_equal(g, ow.sel):
+                        assert stats[wi]["keys_read"] == ow.keys_read and stats[wi]["work"] == ow.work
                     if N == 0:
                         assert lse[wi] == -np.inf and not out[wi].any()
                         continue
-                    o_out, o_lse = O.attend(Kd, Vd, Qh[b, hq, i], ow.sel, C, ot.n_nodes[1], beta)
+                    # the oracle's attention over the GPU's selection
+                    o_out, o_lse = O.attend(Kd, Vd, Qh[b, hq, i], g, C, ot.n_nodes[1], beta)
                     tol = 1e-5 if K.dtype == torch.float32 else 3e-3
                     assert_attention_close(out[wi], lse[wi], o_out, o_lse, tol)
                     if K.dtype == torch.bfloat16:
                         assert_bf16_output_close(out_c[wi], o_out)
+    assert_partings_bounded(parted, walks)
     tree.close()
 
 
@@ -395,6 +416,11 @@ class _Sel:
         self.sel, self.tie_gap, self.tie_sum = sel, gap, sd
 
 
+def _softmax(s):
+    e = np.exp(s - s.max())
+    return e / e.sum()
+
+
 @pytest.mark.parametrize("N,d,dtype,Hq,nq", [(4096, 64, torch.float32, 1, 8), (3001, 128, torch.bfloat16, 4, 2),
                                              (200000, 64, torch.float32, 2, 2), (65536, 128, torch.bfloat16, 4, 8)])
 def test_dense_scan_matches_oracle(N, d, dtype, Hq, nq):
@@ -403,6 +429,7 @@ def test_dense_scan_matches_oracle(N, d, dtype, Hq, nq):
     beta = 1 / np.sqrt(d)
     tree = Z.Tree(K, V, refs, N, 8, 3, beta)
     Qh = host64(Q)
+    parted = walks = 0
     for mode, p, k in ((O.TOP_P, 0.9, 0), (O.TOP_P, 0.5, 0), (O.TOP_P, 1.0, 0), (O.TOP_K, 0, 16), (O.TOP_K, 0, 1)):
         sel, cnt = tree.dense_scan(Q, mode, p, k)
         tree.sync_status()
@@ -413,7 +440,10 @@ def test_dense_scan_matches_oracle(N, d, dtype, Hq, nq):
                 for i in range(nq):
                     wi = (b * Hq + hq) * nq + i
                     s, gap, sd = O.dense_scan(Kd, Qh[b, hq, i], beta, mode, p, k)
-                    compare_selection(sel, cnt, {wi: _Sel(s, gap, sd)})
+                    parted += len(compare_selection(sel, cnt, {wi: _Sel(s, gap, sd)},
+                                                    one_level_valid(_softmax(beta * Kd @ Qh[b, hq, i]), mode, p, k)))
+                    walks += 1
+    assert_partings_bounded(parted, walks)
     tree.close()
 
 
@@ -430,6 +460,7 @@ def test_chunk_mass_matches_oracle(N, d, dtype, Hq, nq, group):
     beta = 1 / np.sqrt(d)
     tree = Z.Tree(K, V, refs, N, 8, 3, beta)
     Qh = host64(Q)
+    parted = walks = 0
     for p in (0.9, 0.5, 1.0):
         sel, cnt, n_chunks = tree.chunk_mass(Q, group, p)
         tree.sync_status()
@@ -442,7 +473,12 @@ def test_chunk_mass_matches_oracle(N, d, dtype, Hq, nq, group):
                     wi = (b * Hq + hq) * nq + i
                     s, nc, gap, sd = O.chunk_mass(Kd, Qh[b, hq, i], beta, group, p)
                     assert nc == n_chunks
-                    compare_selection(sel, cnt, {wi: _Sel(s, gap, sd)})
+                    e = _softmax(beta * Kd @ Qh[b, hq, i])
+                    m = np.add.reduceat(e, np.arange(0, N, group))
+                    parted += len(compare_selection(sel, cnt, {wi: _Sel(s, gap, sd)},
+                                                    one_level_valid(m, O.TOP_P, p, 0)))
+                    walks += 1
+    assert_partings_bounded(parted, walks)
     if group == 1:
         s1, c1 = tree.dense_scan(Q, O.TOP_P, 0.9, 0)
         s2, c2, _ = tree.chunk_mass(Q, 1, 0.9)

@@ -17,7 +17,8 @@ import pytest
 import torch
 
 import oracle as O
-from helpers import assert_attention_close, compare_selection, host64, near_tie
+from helpers import (assert_attention_close, assert_partings_bounded, compare_selection, host64, near_tie,
+                     tree_walk_valid)
 
 pytestmark = pytest.mark.gpu
 
@@ -77,18 +78,21 @@ def test_tensor_core_search_matches_oracle(mode, p, k, N):
     Qh = host64(Q).reshape(-1, D)
     G = (HQ // H) * NQ
     otrees = [O.build_tree(host64(K[0, h, :N]), host64(refs[h]), C, DEPTH, BETA, store=O.STORE_F32) for h in range(H)]
-    checked = 0
+    checked = parted = 0
+    Kh = [host64(K[0, h, :N]) for h in range(H)]
+    Vh = [host64(V[0, h, :N]) for h in range(H)]
     for wi in sample_walks():
         h = wi // G
         ow = O.search(otrees[h], Qh[wi], mode, p, k, 64)
-        if compare_selection(sel_h, cnt_h, {wi: ow}):
-            continue
-        assert stats[wi]["work"] == ow.work and stats[wi]["keys_read"] == ow.keys_read
-        o_out, o_lse = O.attend(host64(K[0, h, :N]), host64(V[0, h, :N]), Qh[wi], ow.sel, C,
-                                otrees[h].n_nodes[1], BETA)
+        if compare_selection(sel_h, cnt_h, {wi: ow}, tree_walk_valid(otrees[h], Qh[wi], mode, p, k, 64)):
+            parted += 1
+        else:
+            assert stats[wi]["work"] == ow.work and stats[wi]["keys_read"] == ow.keys_read
+        # the oracle's attention over the GPU's selection
+        o_out, o_lse = O.attend(Kh[h], Vh[h], Qh[wi], sel_h[wi, : cnt_h[wi]], C, otrees[h].n_nodes[1], BETA)
         assert_attention_close(out[wi], lse[wi], o_out, o_lse, 3e-3, f"walk {wi}")
         checked += 1
-    assert checked > 0.9 * len(sample_walks())
+    assert_partings_bounded(parted, checked, "tensor-core scoring")
 
     # every level went through a tensor-core path (dense, or sparse above 8,192 nodes)
     tree.profile(True)
@@ -106,6 +110,10 @@ def test_tensor_core_search_matches_oracle(mode, p, k, N):
     for wi in differ:
         ow = O.search(otrees[wi // G], Qh[wi], mode, p, k, 64)
         assert near_tie(ow), f"walk {wi}: tensor-core and CUDA-core selections differ away from a tie"
-    print(f"tensor-core scoring: {checked} sampled walks match the oracle; "
+        valid = tree_walk_valid(otrees[wi // G], Qh[wi], mode, p, k, 64)
+        for s, c in ((sel_h, cnt_h), (sel2, cnt2)):
+            assert valid(wi, tuple(int(x) for x in s[wi, : c[wi]])), f"walk {wi}: not an admissible walk"
+    assert_partings_bounded(len(differ), sel_h.shape[0], "tensor-core vs CUDA-core scoring")
+    print(f"tensor-core scoring: {checked} sampled walks checked, {parted} part from the oracle; "
           f"{len(differ)} of {sel_h.shape[0]} walks part from the CUDA-core path, all at oracle near-ties")
     tree.close()
