@@ -144,6 +144,20 @@ int zha_build(const zha_config *cfg, void *K, void *V, const float *refs, long l
 int zha_append(zha_tree *tree, const void *k_new, const void *v_new, void *stream);
 
 /*
+ * zha_rebuild: summarize every level of every tree again, in place, from the
+ * first n keys of the cache and the reference queries as they are now in device
+ * memory. [P1] "What does a node summarize?" and "How is the tree built?" (the
+ * same summaries as zha_build); [P1] "Does the model have to be retrained?": the
+ * reference queries are learned, and each update of them (made in place in the
+ * refs array the tree was built with) needs the summaries made again.
+ * The result equals zha_build over the same keys and refs, bit for bit. The
+ * node storage is reused: nothing is allocated, and the call only launches the
+ * build kernels (level 1, then each level from the one below, on `stream`).
+ * Errors: ZHA_ERR_INVALID (NULL tree), ZHA_ERR_CUDA.
+ */
+int zha_rebuild(zha_tree *tree, void *stream);
+
+/*
  * zha_search: walk every query down its tree ([P1] "Run a small tree yourself",
  * route; "How does top-p differ from top-K?").
  *   1. The frontier starts as every node of the start level (see top_width).
@@ -240,11 +254,13 @@ int zha_chunk_mass(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_hea
  * teacher splits it as the dense attention mass under each node, over the
  * C^l * n_l keys the level covers. loss = mean over the walks of the sum over
  * levels of KL(teacher || tree); grad = d loss / d refs, for the refs the tree
- * was built with (rebuild with zha_build after updating them).
+ * was built with (after updating them in place, zha_rebuild makes the nodes again).
  * Q:    [B][H_q][n_q][d] of q_dtype; at most 32 walks per tree.
  * loss: device float[1]; grad: device float [H_kv][R][d] (both overwritten).
  * Scratch of about 4 * walks * (n + 4 * n_1) + 4 * trees * R * (d + 1) * (sum of
- * the level sizes) bytes is allocated on `stream` and freed there.
+ * the level sizes) bytes is taken from the tree's second scratch block (the one
+ * zha_dense_scan and zha_chunk_mass use), grown with cudaMalloc when too small
+ * and kept for later calls.
  * Errors: ZHA_ERR_INVALID, ZHA_ERR_OOM, ZHA_ERR_CUDA.
  */
 int zha_ref_grad(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q, float *loss, float *grad,
@@ -341,9 +357,10 @@ int zha_sync_status(zha_tree *tree, void *stream);
  * d = 128; 32 MiB holds about 21,000 walks at d = 128, 40,000 at d = 64 and
  * 8,000 at d = 256); a call needing more than 32 MiB fails with
  * ZHA_ERR_CAPACITY and a message giving both sizes, launching nothing.
- * First call: on each device, the first call looks the array's device address up
- * (cudaGetSymbolAddress, with the tree's device current); make that first call
- * before any stream capture.
+ * Every call looks the array's device address up (cudaGetSymbolAddress, with
+ * the tree's device current), so the address stays right after a context reset;
+ * the first call on a device may load the library's module, so make it before
+ * any stream capture.
  * Sharing: every call on a device uses the same array, and each call overwrites
  * what the last one left there. Calls that can overlap on the GPU (different
  * streams, different trees, or different host threads without ordering) race on

@@ -517,3 +517,71 @@ def test_ref_grad_matches_oracle(dtype, d, C, depth):
         scale = max(1e-6, np.abs(grads[h]).max())
         assert np.abs(grad[h] - grads[h]).max() <= 2e-3 * scale, (h, np.abs(grad[h] - grads[h]).max(), scale)
     tree.close()
+
+
+def test_rebuild_after_refs_update_equals_build():
+    """zha_rebuild after the refs were changed in place equals a fresh build with
+    the new refs, bit for bit, and the oracle built with them."""
+    Z = zha()
+    N, C, depth, d, R = 3000, 8, 3, 128, 8
+    K, V, refs, Q = _tiny(N, C=C, depth=depth, d=d, R=R, B=2, H=2, Hq=4, nq=2, dtype=torch.bfloat16, seed=21)
+    beta = 1 / np.sqrt(d)
+    tree = Z.Tree(K, V, refs, N, C, depth, beta)
+    g = torch.Generator(device="cuda").manual_seed(22)
+    refs.mul_(0.5).add_(torch.randn(refs.shape, generator=g, device="cuda"))  # in place: the tree keeps the pointer
+    launches = Z.kernel_launches()
+    tree.rebuild()
+    assert Z.kernel_launches() - launches == depth  # one build launch per level, nothing else
+    fresh = Z.Tree(K, V, refs.clone(), N, C, depth, beta)
+    for l in range(1, depth + 1):
+        a, n = tree.level(l)
+        b, m = fresh.level(l)
+        assert n == m and torch.equal(a[:, :n], b[:, :m])
+    ot = O.build_tree(host64(K[1, 1, :N]), host64(refs[1]), C, depth, beta, store=O.STORE_F32)
+    for l in range(1, depth + 1):
+        gl, n = gpu_level(tree, l, 3)
+        assert_nodes_close(gl, *ot.level(l), R, d)
+    tree.close()
+    fresh.close()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_reference_learning_loop_follows_the_cpu_reference(dtype):
+    """Gradient descent on the references on the GPU (zha_ref_grad, an in-place
+    update, zha_rebuild) follows the CPU reference's descent (autograd in double
+    precision) step by step, and lowers the loss."""
+    from oracle import ref_learning as RL
+
+    Z = zha()
+    B, H, R, Hq, nq, d, C, depth = 1, 2, 3, 4, 4, 64, 4, 3
+    N = C ** depth * 2 + 37
+    K, V, refs, Q = _tiny(N, C=C, d=d, R=R, B=B, H=H, Hq=Hq, nq=nq, dtype=dtype, seed=31)
+    beta, lr, steps = 0.3, 0.5, 6
+    refs0 = refs.clone()
+    tree = Z.Tree(K, V, refs, N, C, depth, beta)
+    gpu = []
+    for _ in range(steps):
+        loss, grad = tree.ref_grad(Q)
+        gpu.append(float(loss.item()))
+        refs.sub_(lr * grad)
+        tree.rebuild()
+    loss, _ = tree.ref_grad(Q)
+    gpu.append(float(loss.item()))
+    tree.sync_status()
+    tree.close()
+    # the GPU loss is the mean over the walks of both trees (equal walks per tree),
+    # so its gradient for head h is 1/H of that head's own: the same trajectory as
+    # per-head descent with step lr / H
+    group = Hq // H
+    Qh = host64(Q)
+    per_head = []
+    for h in range(H):
+        q = torch.from_numpy(Qh[0, h * group: (h + 1) * group].reshape(-1, d))
+        _, losses = RL.learn_refs(torch.from_numpy(host64(K[0, h, :N])), torch.from_numpy(host64(refs0[h])), q, C,
+                                  depth, beta, steps, lr / H)
+        per_head.append(losses)
+    ref = np.mean(np.array(per_head), axis=0)
+    err = np.abs(np.array(gpu) - ref) / np.maximum(1.0, np.abs(ref))
+    print("losses (GPU, CPU reference):", list(zip(np.round(gpu, 6), np.round(ref, 6))))
+    assert err.max() <= 1e-4, (gpu, ref.tolist())
+    assert gpu[-1] < gpu[0]

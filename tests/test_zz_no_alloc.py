@@ -5,10 +5,12 @@ that gives all GPU memory to its own pool at start-up, a latency-critical loop t
 cannot take the synchronisation cudaMalloc / cudaFree may cause) call
 zha_attend_noalloc instead of zha_attend: same arguments, same kernels, with the
 scratch taken from a 32 MiB static device array of the library. These tests call
-it through the C ABI and check, on two calls in a row with different walk counts,
-selections and output types, that it gives what zha_attend gives, that the
-second call changes the device's free memory by nothing, and that a call needing
-more than the array holds is refused before anything is launched.
+it through the C ABI and check, on calls in a row with different walk counts,
+selections and output types, that it gives what zha_attend gives, that the calls
+after the first change the device's free memory by nothing, and that a call
+needing more than the array holds is refused before anything is launched. The
+third call has more than 2,048 walks, which takes the attention's separate plan
+kernel, right after smaller calls have left their plans in the array.
 
 The file is named to be collected last, so that a run stopping at the first
 failure has run every other test before it.
@@ -67,9 +69,10 @@ def test_noalloc_matches_attend_on_two_calls():
     inp = S.draw(w, device="cuda")
     tree = Z.Tree(inp.K, inp.V, inp.refs, w.n_keys, w.chunk, w.depth, w.beta, w.top_width)
     atol = attn_tol(w)
-    calls = [  # (queries per head, mode, p, k, output dtype): the two calls differ in every one
+    calls = [  # (queries per head, mode, p, k, output dtype): consecutive calls differ in every one
         (1, Z.TOP_P, 0.9, 0, torch.float32),
         (3, Z.TOP_K, 0.0, 8, torch.bfloat16),
+        (48, Z.TOP_P, 0.9, 0, torch.float32),  # 3,072 walks: the plan-kernel path
     ]
     for i, (n_q, mode, p, k, out_dtype) in enumerate(calls):
         Q = queries(w, inp, n_q)

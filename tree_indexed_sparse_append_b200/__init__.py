@@ -28,7 +28,7 @@ TOP_P, TOP_K = 0, 1
 SYMBOLS = ("zha_build", "zha_append", "zha_search", "zha_attend", "zha_reserve", "zha_level",
            "zha_num_keys", "zha_depth", "zha_sync_status", "zha_destroy", "zha_last_error", "zha_version",
            "zha_profile", "zha_profile_read", "zha_kernel_launches", "zha_last_search_info",
-           "zha_dense_scan", "zha_attend_noalloc", "zha_chunk_mass", "zha_ref_grad")
+           "zha_dense_scan", "zha_attend_noalloc", "zha_chunk_mass", "zha_ref_grad", "zha_rebuild")
 KERNEL_KINDS = ("build", "append", "search_init", "score", "select", "attend_plan", "attend_partial",
                 "attend_combine", "score_tc")
 
@@ -76,6 +76,7 @@ def lib():
         vp, i, ll, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
         L.zha_build.argtypes = [ctypes.POINTER(Config), vp, vp, vp, ll, vp, ctypes.POINTER(vp)]
         L.zha_append.argtypes = [vp, vp, vp, vp]
+        L.zha_rebuild.argtypes = [vp, vp]
         L.zha_search.argtypes = [vp, vp, i, i, i, i, f, i, vp, vp, i, vp, vp]
         L.zha_attend.argtypes = [vp, vp, i, i, i, vp, vp, i, vp, i, vp, vp]
         L.zha_attend_noalloc.argtypes = [vp, vp, i, i, i, vp, vp, i, vp, i, vp, vp]
@@ -203,6 +204,11 @@ class Tree:
         if k_new.shape != (B, H, d) or v_new.shape != (B, H, d) or k_new.dtype != self.K.dtype or v_new.dtype != self.K.dtype:
             raise ValueError("k_new and v_new must be [B][H_kv][d] of the cache dtype")
         _check(lib().zha_append(self._h, _dev(k_new, "k_new"), _dev(v_new, "v_new"), _stream(stream)))
+
+    def rebuild(self, stream=None) -> None:
+        """Summarize every level again in place from the cache and the current
+        refs (after the refs were updated in place); allocates nothing."""
+        _check(lib().zha_rebuild(self._h, _stream(stream)))
 
     def search(self, Q: torch.Tensor, mode: int = TOP_P, p: float = 0.9, k: int = 1, max_sel: int | None = None,
                with_stats: bool = False, out=None, stream=None):

@@ -327,6 +327,14 @@ int zha_append(zha_tree *t, const void *k_new, const void *v_new, void *stream) 
     return ZHA_OK;
 }
 
+int zha_rebuild(zha_tree *t, void *stream) {
+    if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    for (int l = 1; l <= t->max_depth; ++l)
+        ZHA_CUDA(zha::launch_build_level(t, l, 0, t->n_nodes[l], st), "launching the rebuild");
+    return ZHA_OK;
+}
+
 static int check_queries(const zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q,
                          long long *W, int *G) {
     if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");
@@ -388,8 +396,10 @@ int zha_attend(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads, int
     return ZHA_OK;
 }
 
+}  // extern "C"
+
 // Grows the tree's full-scan scratch to at least `need` bytes.
-static int grow_dense_scratch(zha_tree *t, size_t need) {
+int zha::grow_dense_scratch(zha_tree *t, size_t need) {
     if (need <= t->dws_bytes) return ZHA_OK;
     if (t->dws) cudaFree(t->dws);
     t->dws = nullptr;
@@ -402,6 +412,8 @@ static int grow_dense_scratch(zha_tree *t, size_t need) {
     t->dws_bytes = need;
     return ZHA_OK;
 }
+
+extern "C" {
 
 int zha_chunk_mass(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q, int group, float p,
                    int *sel, int *count, int max_sel, void *stream) {
@@ -419,7 +431,7 @@ int zha_chunk_mass(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads,
     const size_t o_S = align_up(sizeof(float) * W * t->cfg.d);
     const size_t o_Sc = o_S + align_up(sizeof(float) * W * N);
     const size_t o_gk = o_Sc + align_up(sizeof(float) * W * nch);
-    rc = grow_dense_scratch(t, o_gk + align_up(sizeof(uint32_t) * W * nch));
+    rc = zha::grow_dense_scratch(t, o_gk + align_up(sizeof(uint32_t) * W * nch));
     if (rc) return rc;
     char *b = static_cast<char *>(t->dws);
     ZHA_CUDA(zha::launch_chunk_mass(t, Q, q_dtype, G, W, group, p, sel, count, max_sel, reinterpret_cast<float *>(b),
@@ -448,7 +460,7 @@ int zha_dense_scan(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads,
     const long long N = t->n > 0 ? t->n : 1;
     const size_t need = align_up(sizeof(float) * W * t->cfg.d) + align_up(sizeof(float) * W * N) +
                         align_up(sizeof(uint32_t) * W * N);
-    rc = grow_dense_scratch(t, need);
+    rc = zha::grow_dense_scratch(t, need);
     if (rc) return rc;
     char *b = static_cast<char *>(t->dws);
     float *qf = reinterpret_cast<float *>(b);

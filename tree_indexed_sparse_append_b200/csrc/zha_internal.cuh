@@ -265,6 +265,9 @@ cudaError_t launch_score_tc_sparse(const zha_tree *t, int level, int G, const vo
                                    long long Sstride, cudaStream_t st);
 // Records an error message for zha_last_error (this host thread); returns code.
 int set_error(int code, const char *msg);
+// Grows the tree's second scratch block (full-scan indexer, chunk-mass profile,
+// split-loss gradient) to at least `need` bytes; returns a ZHA_ status.
+int grow_dense_scratch(zha_tree *t, size_t need);
 
 // kernel launchers (return cudaError_t of the launch)
 cudaError_t launch_build_level(const zha_tree *t, int level, long long j0, long long j1,

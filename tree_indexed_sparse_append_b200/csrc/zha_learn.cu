@@ -356,14 +356,12 @@ extern "C" int zha_ref_grad(zha_tree *t, const void *Q, zha_dtype q_dtype, int n
     const size_t gbytes = o - off[6];
     o = al(o);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    void *ws = nullptr;
-    cudaError_t e = cudaMallocAsync(&ws, o, st);
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        return set_error(ZHA_ERR_OOM, "allocating the split-loss scratch");
-    }
-    char *b = static_cast<char *>(ws);
-    e = cudaMemsetAsync(b + off[6], 0, gbytes, st);
+    // the tree's second scratch block, shared with the full-scan indexer (grown
+    // when too small, then reused by later calls)
+    const int rc = zha::grow_dense_scratch(t, o);
+    if (rc) return rc;
+    char *b = static_cast<char *>(t->dws);
+    cudaError_t e = cudaMemsetAsync(b + off[6], 0, gbytes, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(loss, 0, sizeof(float), st);
     if (e == cudaSuccess) e = cudaMemsetAsync(grad, 0, sizeof(float) * (size_t)c.n_kv_heads * c.R * c.d, st);
     if (e == cudaSuccess && t->n > 0) {
@@ -373,7 +371,6 @@ extern "C" int zha_ref_grad(zha_tree *t, const void *Q, zha_dtype q_dtype, int n
             default: e = zha::learn_d<256>(t, Q, q_dtype, (int)G, W, loss, grad, b, off, st); break;
         }
     }
-    cudaFreeAsync(ws, st);
     if (e != cudaSuccess) return set_error(ZHA_ERR_CUDA, cudaGetErrorString(e));
     return ZHA_OK;
 }

@@ -11,39 +11,33 @@
 // that loads the library holds that array until the process exits.
 //
 // In host code the array's name is only a host-side stand-in, not a device
-// address, so the address is looked up with cudaGetSymbolAddress, once per
-// device with that device current, and that address is what the kernels get.
+// address, so the address is looked up with cudaGetSymbolAddress, with the
+// tree's device current, and that address is what the kernels get. The lookup
+// runs on every call (it allocates nothing): a cached address would go stale if
+// the device's primary context were torn down and made again (cudaDeviceReset),
+// which loads the module, and the array, at a new address.
 // The kernels themselves are zha_attend's; only where their scratch lives differs.
 #include <cstdio>
-#include <mutex>
 
 #include "zha_internal.cuh"
 
 namespace {
 
 constexpr size_t ZHA_NOALLOC_SCRATCH_BYTES = size_t(32) << 20;  // 32 MiB per device
-constexpr int MAX_DEVICES = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[ZHA_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_addr_mu;
-void *g_addr[MAX_DEVICES];  // device address of g_noalloc_scratch, per device
-
-// Device address of the array on the current device; looked up on the first call.
-int scratch_address(int dev, void **out) {
-    std::lock_guard<std::mutex> lock(g_addr_mu);
-    if (!g_addr[dev]) {
-        void *p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess || !p) {
-            char msg[256];
-            snprintf(msg, sizeof msg, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
-            cudaGetLastError();
-            return zha::set_error(ZHA_ERR_CUDA, msg);
-        }
-        g_addr[dev] = p;
+// Device address of the array on the current device.
+int scratch_address(void **out) {
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+        char msg[256];
+        snprintf(msg, sizeof msg, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
+        cudaGetLastError();
+        return zha::set_error(ZHA_ERR_CUDA, msg);
     }
-    *out = g_addr[dev];
+    *out = p;
     return ZHA_OK;
 }
 
@@ -82,9 +76,8 @@ extern "C" int zha_attend_noalloc(zha_tree *t, const void *Q, zha_dtype q_dtype,
         return zha::set_error(ZHA_ERR_CUDA, "cudaGetDevice failed");
     }
     if (dev != t->device) return zha::set_error(ZHA_ERR_INVALID, "the current device is not the tree's device");
-    if (dev < 0 || dev >= MAX_DEVICES) return zha::set_error(ZHA_ERR_INVALID, "device index beyond 63");
     void *base = nullptr;
-    int rc = scratch_address(dev, &base);
+    int rc = scratch_address(&base);
     if (rc) return rc;
 
     zha::Scratch s{};
@@ -93,12 +86,13 @@ extern "C" int zha_attend_noalloc(zha_tree *t, const void *Q, zha_dtype q_dtype,
     // plan kernel for large calls) and computes every offset and item length it
     // reads, so what an earlier call left in the array needs no clearing here.
 
-    // The profiler's CUDA events are created on demand; keep it out of this call.
-    zha_profiler *prof = t->prof;
-    t->prof = nullptr;
-    e = zha::launch_attend(t, s, Q, q_dtype, (int)G, W, sel, sel_count, max_sel, out, out_dtype, lse,
+    // The profiler's CUDA events are created on demand, so this call is not
+    // profiled: the launches get a copy of the handle without its profiler, and
+    // the caller's tree is never modified (other host threads may be using it).
+    zha_tree unprofiled = *t;
+    unprofiled.prof = nullptr;
+    e = zha::launch_attend(&unprofiled, s, Q, q_dtype, (int)G, W, sel, sel_count, max_sel, out, out_dtype, lse,
                            static_cast<cudaStream_t>(stream));
-    t->prof = prof;
     if (e != cudaSuccess) {
         char msg[256];
         snprintf(msg, sizeof msg, "launching the attention: %s", cudaGetErrorString(e));
