@@ -316,6 +316,20 @@ int zha_profile_read(zha_tree *tree, zha_kernel_time *out, void *stream);
 /* Kernels launched by this library in this process, all trees together. */
 long long zha_kernel_launches(void);
 
+/*
+ * zha_test_wait_limit: test hook for the bounded waits of the tensor-core scorer
+ * (prefill scoring, trees of at least 1,024 bf16 walks at d = 128). Every wait
+ * of those kernels on a copy or an MMA gives up after wait_ns nanoseconds
+ * (0 restores the default of 1 s), records ZHA_ERR_TIMEOUT for zha_sync_status,
+ * waits (again bounded) for the copies and MMAs its CTA issued, frees its tensor
+ * memory and returns. With stall = 1, every later dense scoring launch of this
+ * tree first waits on a barrier that nothing arrives at, before issuing any copy
+ * or MMA, so that wait runs out: the results of that search are undefined and
+ * zha_sync_status returns ZHA_ERR_TIMEOUT. stall = 0 turns it off. Not for
+ * production use.
+ */
+int zha_test_wait_limit(zha_tree *tree, long long wait_ns, int stall);
+
 /* Size of the frontiers of the last zha_search on this tree. */
 typedef struct {
     int start_level;

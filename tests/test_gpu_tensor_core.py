@@ -117,3 +117,39 @@ def test_tensor_core_search_matches_oracle(mode, p, k, N):
     print(f"tensor-core scoring: {checked} sampled walks checked, {parted} part from the oracle; "
           f"{len(differ)} of {sel_h.shape[0]} walks part from the CUDA-core path, all at oracle near-ties")
     tree.close()
+
+
+def test_bounded_wait_runs_out_and_is_reported():
+    """The tensor-core scorer's waits are bounded. With the test hook on, each
+    CTA's first wait (before any copy or MMA) is on a barrier that nothing
+    arrives at; it gives up after 2 ms, the search reports ZHA_ERR_TIMEOUT through
+    zha_sync_status, and once the hook is off the same tree searches correctly
+    again (the context is still usable)."""
+    Z = zha()
+    N = 16427
+    K, V, refs, Q = inputs(N, seed=11)
+    tree = Z.Tree(K, V, refs, N, C, DEPTH, BETA)
+    max_sel = N // C
+    sel_a, cnt_a, _ = tree.search(Q, Z.TOP_P, 0.9, 0, max_sel=max_sel)
+    tree.sync_status()
+    sel_a, cnt_a = sel_a.cpu().numpy(), cnt_a.cpu().numpy()
+
+    tree.test_wait_limit(2_000_000, stall=True)
+    tree.profile(True)
+    tree.search(Q, Z.TOP_P, 0.9, 0, max_sel=max_sel)
+    kinds = tree.profile_read()
+    tree.profile(False)
+    assert kinds["score_tc"][0] > 0  # the dense tensor-core scorer ran
+    with pytest.raises(Z.ZhaError) as e:
+        tree.sync_status()
+    assert e.value.code == Z.ERR_TIMEOUT
+    tree.sync_status()  # the status word was cleared
+
+    tree.test_wait_limit(0, stall=False)
+    sel_b, cnt_b, _ = tree.search(Q, Z.TOP_P, 0.9, 0, max_sel=max_sel)
+    tree.sync_status()
+    sel_b, cnt_b = sel_b.cpu().numpy(), cnt_b.cpu().numpy()
+    assert np.array_equal(cnt_a, cnt_b)
+    for w in range(len(cnt_a)):
+        assert np.array_equal(sel_a[w, : cnt_a[w]], sel_b[w, : cnt_b[w]])
+    tree.close()

@@ -28,7 +28,8 @@ TOP_P, TOP_K = 0, 1
 SYMBOLS = ("zha_build", "zha_append", "zha_search", "zha_attend", "zha_reserve", "zha_level",
            "zha_num_keys", "zha_depth", "zha_sync_status", "zha_destroy", "zha_last_error", "zha_version",
            "zha_profile", "zha_profile_read", "zha_kernel_launches", "zha_last_search_info",
-           "zha_dense_scan", "zha_attend_noalloc", "zha_chunk_mass", "zha_ref_grad", "zha_rebuild")
+           "zha_dense_scan", "zha_attend_noalloc", "zha_chunk_mass", "zha_ref_grad", "zha_rebuild",
+           "zha_test_wait_limit")
 KERNEL_KINDS = ("build", "append", "search_init", "score", "select", "attend_plan", "attend_partial",
                 "attend_combine", "score_tc")
 
@@ -77,6 +78,7 @@ def lib():
         L.zha_build.argtypes = [ctypes.POINTER(Config), vp, vp, vp, ll, vp, ctypes.POINTER(vp)]
         L.zha_append.argtypes = [vp, vp, vp, vp]
         L.zha_rebuild.argtypes = [vp, vp]
+        L.zha_test_wait_limit.argtypes = [vp, ll, i]
         L.zha_search.argtypes = [vp, vp, i, i, i, i, f, i, vp, vp, i, vp, vp]
         L.zha_attend.argtypes = [vp, vp, i, i, i, vp, vp, i, vp, i, vp, vp]
         L.zha_attend_noalloc.argtypes = [vp, vp, i, i, i, vp, vp, i, vp, i, vp, vp]
@@ -321,6 +323,12 @@ class Tree:
         _check(lib().zha_last_search_info(self._h, ctypes.byref(info), _stream(stream)))
         return {"start_level": info.start_level, "union_nodes": list(info.union_nodes),
                 "walk_nodes": list(info.walk_nodes)}
+
+    def test_wait_limit(self, wait_ns: int, stall: bool = False) -> None:
+        """Test hook: the tensor-core scorer's waits give up after wait_ns (0: the
+        default 1 s); with stall, its launches first wait on a barrier nothing
+        arrives at, so the search reports ZHA_ERR_TIMEOUT."""
+        _check(lib().zha_test_wait_limit(self._h, int(wait_ns), 1 if stall else 0))
 
     def sync_status(self, stream=None) -> None:
         _check(lib().zha_sync_status(self._h, _stream(stream)))

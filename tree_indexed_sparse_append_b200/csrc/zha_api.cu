@@ -540,6 +540,14 @@ int zha_profile_read(zha_tree *t, zha_kernel_time *out, void *stream) {
 
 long long zha_kernel_launches(void) { return g_launches.load(); }
 
+int zha_test_wait_limit(zha_tree *t, long long wait_ns, int stall) {
+    if (!t) return fail(ZHA_ERR_INVALID, "tree is NULL");
+    if (wait_ns < 0) return fail(ZHA_ERR_INVALID, "wait_ns must be >= 0");
+    t->tc_wait_ns = (unsigned long long)wait_ns;
+    t->tc_stall = stall ? 1 : 0;
+    return ZHA_OK;
+}
+
 int zha_last_search_info(zha_tree *t, zha_search_info *out, void *stream) {
     if (!t || !out) return fail(ZHA_ERR_INVALID, "NULL argument");
     memset(out, 0, sizeof *out);

@@ -198,6 +198,8 @@ struct zha_tree {
 
     // diagnostics
     struct zha_profiler *prof;  // NULL unless zha_profile(tree, 1)
+    unsigned long long tc_wait_ns;  // limit of the tensor-core scorer's waits (0: 1 s)
+    int tc_stall;                   // test hook of zha_test_wait_limit
     long long last_W;
     int last_G, last_start, last_max_sel;
 };

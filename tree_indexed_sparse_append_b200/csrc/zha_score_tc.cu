@@ -57,10 +57,10 @@ constexpr int TC_BTILE = 3 * TC_PART + TC_N * 4;     // hi, mid, lo, biases
 constexpr int TC_ATILE = TC_M * TC_K * 2;
 constexpr int TC_MT = 2;                             // A tiles (of 128 walks) per CTA
 constexpr int TC_SLOTS = 4;                          // B part slots in shared memory
-constexpr int TC_SMEM = TC_MT * TC_ATILE + TC_SLOTS * TC_PART + 128;  // + barriers, TMEM address, flag
+constexpr int TC_SMEM = TC_MT * TC_ATILE + TC_SLOTS * TC_PART + 256;  // + barriers, TMEM address, flag
 constexpr int TC_TMEM_COLS = 512;                    // TC_MT x 2 fp32 accumulators of 128 columns
 constexpr int TC_THREADS = 9 * 32;                   // 8 epilogue warps + 1 producer warp
-constexpr unsigned long long TC_WAIT_NS = 1000000000ull;  // a wait gives up after 1 s
+constexpr unsigned long long TC_WAIT_NS = 1000000000ull;  // a wait gives up after 1 s (unless the tree sets less)
 
 // byte offset of element (row, k) in a 128-row K-major tile without swizzle:
 // 8-row x 16-byte core matrices, consecutive along K (128 B apart), 8-row groups
@@ -107,11 +107,11 @@ __device__ __forceinline__ unsigned long long global_ns() {
     return t;
 }
 
-// bounded wait; false when it gave up
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase) {
+// bounded wait (at most limit_ns of %globaltimer); false when it gave up
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, unsigned long long limit_ns) {
     if (mbar_try_wait(bar, phase)) return true;
     const unsigned long long t0 = global_ns();
-    while (global_ns() - t0 < TC_WAIT_NS)
+    while (global_ns() - t0 < limit_ns)
         if (mbar_try_wait(bar, phase)) return true;
     return false;
 }
@@ -246,6 +246,8 @@ struct ScoreTcArgs {
     float *S;
     long long Sstride;
     int *status;
+    unsigned long long wait_ns;  // limit of every wait
+    int stall;                   // test hook: the producer first waits on a barrier nothing arrives at
 };
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
@@ -263,9 +265,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(ScoreTcArgs a) 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TC_MT * TC_ATILE + TC_SLOTS * TC_PART);
     // bars 0-3: slot filled; 4-7: slot's MMAs done; 8-9: accumulator buffer written
     // (MMA commit); 10-11: accumulator buffer read back (8 warps); 12: A tiles
-    // filled; 13: all MMAs done (cleanup)
+    // filled; 13: all MMAs done (cleanup); 16: the test hook's barrier, which
+    // nothing arrives at
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
     volatile int *fail = reinterpret_cast<volatile int *>(bars + 15);
+    const unsigned long long lim = a.wait_ns;
+    auto mbar_wait = [lim](uint32_t bar, uint32_t phase) { return zha::mbar_wait(bar, phase, lim); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long ct = blockIdx.x, t = blockIdx.y;
@@ -275,10 +280,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(ScoreTcArgs a) 
     auto empty = [&](int s) { return smem_u32(bars + 4 + s); };
     auto accf = [&](int b) { return smem_u32(bars + 8 + b); };
     auto accfree = [&](int b) { return smem_u32(bars + 10 + b); };
-    const uint32_t barA = smem_u32(bars + 12), barEnd = smem_u32(bars + 13);
+    const uint32_t barA = smem_u32(bars + 12), barEnd = smem_u32(bars + 13), barStall = smem_u32(bars + 16);
 
     if (tid == 0) {
         *fail = 0;
+        mbar_init(barStall, 1);
         for (int i = 0; i < TC_SLOTS; ++i) {
             mbar_init(full(i), 1);
             mbar_init(empty(i), 1);
@@ -305,20 +311,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(ScoreTcArgs a) 
     if (warp == 8) {
         // producer: one thread issues every copy and MMA
         if (lane == 0) {
-            bool ok = true;
+            // the test hook: a wait that runs out before any copy or MMA is issued
+            bool ok = !a.stall || mbar_wait(barStall, 0);
             long long fills[TC_SLOTS] = {0, 0, 0, 0}, waited[TC_SLOTS] = {0, 0, 0, 0};
-            bool a_waited = false, any_mma = false;
+            bool a_issued = false, a_waited = false, any_mma = false;
             auto fill = [&](long long j) {  // B part j -> slot j % 4
                 const int s = (int)(j & (TC_SLOTS - 1));
                 mbar_expect_tx(full(s), TC_PART);
                 bulk_g2s(smem_u32(sB + s * TC_PART), btree + (j / 3) * TC_BTILE + (j % 3) * TC_PART, TC_PART, full(s));
                 ++fills[s];
             };
-            mbar_expect_tx(barA, TC_MT * TC_ATILE);
-            bulk_g2s(smem_u32(sA), a.atiles + (t * a.mtiles + TC_MT * ct) * TC_ATILE, TC_MT * TC_ATILE, barA);
-            for (long long j = 0; j < TC_SLOTS && j < nparts; ++j) fill(j);
-            if (mbar_wait(barA, 0)) a_waited = true;
-            else ok = false;
+            if (ok) {
+                mbar_expect_tx(barA, TC_MT * TC_ATILE);
+                bulk_g2s(smem_u32(sA), a.atiles + (t * a.mtiles + TC_MT * ct) * TC_ATILE, TC_MT * TC_ATILE, barA);
+                a_issued = true;
+                for (long long j = 0; j < TC_SLOTS && j < nparts; ++j) fill(j);
+                if (mbar_wait(barA, 0)) a_waited = true;
+                else ok = false;
+            }
             for (long long n = 0; ok && n < ntiles; ++n) {
                 const int b = (int)(n & 1);
                 // accumulator buffer b is free once the epilogue of tile n - 2 read it
@@ -364,7 +374,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_tc_kernel(ScoreTcArgs a) 
                 *fail = 1;
                 report(a.status, DEV_TIMEOUT);
                 // let the copies and MMAs in flight finish (bounded waits)
-                if (!a_waited) (void)mbar_wait(barA, 0);
+                if (a_issued && !a_waited) (void)mbar_wait(barA, 0);
                 for (int s = 0; s < TC_SLOTS; ++s)
                     if (fills[s] > waited[s]) (void)mbar_wait(full(s), (uint32_t)((fills[s] - 1) & 1));
                 if (any_mma) {
@@ -518,6 +528,7 @@ struct SparseArgs {
     float *S;
     long long Sstride;
     int *status;
+    unsigned long long wait_ns;  // limit of every wait
 };
 
 constexpr int TS_SMEM = 3 * TC_PART + TC_ATILE + TC_N * 4 + 64;  // B tile, gathered walks, biases, barriers
@@ -543,6 +554,8 @@ __global__ void __launch_bounds__(128, 1) score_tc_sparse_kernel(SparseArgs a) {
     if (count <= 0) return;  // the same for the whole CTA; nothing allocated yet
     const int *list = a.lists + tn * a.G;
     const uint32_t barB = smem_u32(bars), barM = smem_u32(bars + 1);
+    const unsigned long long lim = a.wait_ns;
+    auto mbar_wait = [lim](uint32_t bar, uint32_t phase) { return zha::mbar_wait(bar, phase, lim); };
 
     if (tid == 0) {
         mbar_init(barB, 1);
@@ -695,6 +708,7 @@ cudaError_t launch_score_tc_sparse(const zha_tree *t, int level, int G, const vo
     sa.S = S;
     sa.Sstride = Sstride;
     sa.status = t->d_status;
+    sa.wait_ns = t->tc_wait_ns ? t->tc_wait_ns : TC_WAIT_NS;
     switch (RP) {
         case 4: return launch_sparse_rp<4>(t, sa, st);
         case 8: return launch_sparse_rp<8>(t, sa, st);
@@ -781,6 +795,8 @@ cudaError_t launch_score_tc(const zha_tree *t, int level, int G, unsigned char *
     sa.S = S;
     sa.Sstride = Sstride;
     sa.status = t->d_status;
+    sa.wait_ns = t->tc_wait_ns ? t->tc_wait_ns : TC_WAIT_NS;
+    sa.stall = t->tc_stall;
     switch (RP) {
         case 1: return launch_score_tc_rp<1>(t, sa, st);
         case 2: return launch_score_tc_rp<2>(t, sa, st);
