@@ -9,12 +9,26 @@
 // node j of level l covers nodes C*j .. C*j+C-1 of level l-1, and a node is made
 // when its chunk fills.
 //
-// Mapping: one warp per (node, reference); a block holds the R warps of one
-// node, so the level-1 children (the keys, shared by every reference) are read
-// from HBM once and then from L1. Lane l owns D/32 consecutive columns. The
-// per-child partial dot products are exchanged through shared memory (a
-// [child][lane] tile), summed by the lane that owns the child, and the softmax
-// weights are broadcast back for the weighted key sum. All arithmetic is fp32.
+// Mapping (all arithmetic fp32; the softmax is taken online over batches of
+// children, so a node's children are read once):
+//   build_leaf_kernel   level 1: a warp per node and group of RPW references
+//                       (4 at D = 128: two warps per node at R = 8, the second
+//                       one's key reads hitting L1). Lane l owns D/32
+//                       consecutive columns of each key; the keys of a batch are
+//                       loaded together (all loads in flight at once), each key's
+//                       RPW dot products are summed across the warp by one
+//                       transpose-reduce, and every lane then takes the weights
+//                       of its warp's references by shuffles to accumulate their
+//                       weighted keys in registers.
+//   build_upper_kernel  levels >= 2: one warp per (node, reference), reading
+//                       row r of each child (consecutive warps take the rows of
+//                       one node, so the node is written row after row); the
+//                       batch's child rows are loaded together, their dot
+//                       products summed by one transpose-reduce and shuffled to
+//                       every lane.
+//   build_nodes_kernel  the earlier general kernel, kept as a fallback for an
+//                       unexpected head dimension: a block of R warps per node,
+//                       partial dot products exchanged through shared memory.
 #include "zha_internal.cuh"
 
 namespace zha {
@@ -115,6 +129,260 @@ __global__ void __launch_bounds__(512) build_nodes_kernel(BuildArgs a) {
     chain_done();
 }
 
+// Level-1 nodes: WPN = ceil(R / RPW) warps per node, each taking RPW of its
+// references (RPW a power of two; rows past R are zero and unused); the keys come
+// KB at a time (KB * D / 32 registers of keys per lane: 32, or 16 at D = 64).
+template <typename KT, int D, int RPW>
+__global__ void __launch_bounds__(256, 2) build_leaf_kernel(BuildArgs a) {
+    chain_start();
+    constexpr int EPL = D / 32;
+    constexpr int KB = 32 / EPL < 8 ? 32 / EPL : 8;  // keys per batch
+    constexpr int LG = ilog2(RPW);
+    const int lane = threadIdx.x & 31;
+    const int rr = lane >> (5 - LG);  // reference (of this warp's RPW) whose sums this lane ends with
+    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+    const KT *K = static_cast<const KT *>(a.child);
+    const int wpn = (a.R + RPW - 1) / RPW;
+    const long long witems = a.items * wpn;
+
+    for (long long wi = gw; wi < witems; wi += nw) {
+        const long long item = wi / wpn;
+        const int r0 = (int)(wi - item * wpn) * RPW;
+        const long long t = item / a.per_tree;
+        const long long j = a.j0 + item % a.per_tree;
+        const int h = (int)(t % a.H_kv);
+        float q[RPW][EPL];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) {
+            if (r0 + r < a.R) {
+                load_cached<EPL>(a.refs + ((long long)h * a.R + r0 + r) * D + lane * EPL, q[r]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) q[r][e] = 0.f;
+            }
+        }
+        const KT *keys = K + t * a.child_tree + j * a.C * (long long)D + lane * EPL;
+        float m = -INFINITY, z = 0.f;  // running max and sum of exp, of reference r0 + rr
+        float acc[RPW][EPL];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r)
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[r][e] = 0.f;
+
+        for (int i0 = 0; i0 < a.C; i0 += KB) {
+            float kf[KB][EPL];
+#pragma unroll
+            for (int i = 0; i < KB; ++i) {
+                if (i0 + i < a.C) {
+                    load_cached<EPL>(keys + (long long)(i0 + i) * D, kf[i]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) kf[i][e] = 0.f;
+                }
+            }
+            // s[i]: beta <k_i, q_rr> (lanes of reference rr)
+            float s[KB];
+#pragma unroll
+            for (int i = 0; i < KB; ++i) {
+                float part[RPW];
+#pragma unroll
+                for (int r = 0; r < RPW; ++r) {
+                    float x = 0.f;
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) x = fmaf(kf[i][e], q[r][e], x);
+                    part[r] = x;
+                }
+                const float dot = transpose_reduce<RPW>(part, lane);
+                s[i] = i0 + i < a.C ? a.beta * dot : -INFINITY;
+            }
+            float bm = m;
+#pragma unroll
+            for (int i = 0; i < KB; ++i) bm = fmaxf(bm, s[i]);
+            const float scale = expf(m - bm);  // 0 on the first batch (m = -inf)
+            z *= scale;
+            float wt[KB];
+#pragma unroll
+            for (int i = 0; i < KB; ++i) {
+                wt[i] = expf(s[i] - bm);
+                z += wt[i];
+            }
+            m = bm;
+            // every lane takes each reference's scale and weights from that
+            // reference's lanes and accumulates its columns of the RPW sums
+#pragma unroll
+            for (int r = 0; r < RPW; ++r) {
+                const int src = r << (5 - LG);
+                const float sc = __shfl_sync(FULL, scale, src);
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) acc[r][e] *= sc;
+#pragma unroll
+                for (int i = 0; i < KB; ++i) {
+                    const float w = __shfl_sync(FULL, wt[i], src);
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) acc[r][e] = fmaf(w, kf[i][e], acc[r][e]);
+                }
+            }
+        }
+        // key_r = acc_r / z_r; bias_r = m_r + log z_r - beta <key_r, q_r>
+        float *node = a.out + t * a.out_tree + j * a.NF;
+        float part[RPW];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) {
+            const float zr = __shfl_sync(FULL, z, r << (5 - LG));
+            float x = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+                acc[r][e] = acc[r][e] / zr;
+                x = fmaf(acc[r][e], q[r][e], x);
+            }
+            part[r] = x;
+            if (r0 + r < a.R) {
+                float *row = node + (r0 + r) * D + lane * EPL;
+                if constexpr (EPL % 4 == 0) {
+#pragma unroll
+                    for (int e = 0; e < EPL; e += 4)
+                        *reinterpret_cast<float4 *>(row + e) = make_float4(acc[r][e], acc[r][e + 1], acc[r][e + 2],
+                                                                           acc[r][e + 3]);
+                } else {
+                    *reinterpret_cast<float2 *>(row) = make_float2(acc[r][0], acc[r][1]);
+                }
+            }
+        }
+        const float dq = transpose_reduce<RPW>(part, lane);
+        if (r0 + rr < a.R && (lane & ((32 >> LG) - 1)) == 0)
+            node[a.R * D + r0 + rr] = m + logf(z) - a.beta * dq;
+    }
+    chain_done();
+}
+
+// Levels >= 2, one warp per (node, reference r): row r of each child, CB at a
+// time (CB * D / 32 registers of rows per lane).
+template <int D>
+__global__ void __launch_bounds__(256, 2) build_upper_kernel(BuildArgs a) {
+    chain_start();
+    constexpr int EPL = D / 32;
+    constexpr int CB = 32 / EPL;  // children per batch
+    constexpr int LG = ilog2(CB);
+    const int lane = threadIdx.x & 31;
+    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+    const float *nodes = static_cast<const float *>(a.child);
+    const long long witems = a.items * a.R;
+
+    for (long long wi = gw; wi < witems; wi += nw) {
+        const long long item = wi / a.R;
+        const int r = (int)(wi - item * a.R);
+        const long long t = item / a.per_tree;
+        const long long j = a.j0 + item % a.per_tree;
+        const int h = (int)(t % a.H_kv);
+        float q[EPL];
+        load_cached<EPL>(a.refs + ((long long)h * a.R + r) * D + lane * EPL, q);
+        const float *children = nodes + t * a.child_tree + j * a.C * a.child_stride;
+        float m = -INFINITY, z = 0.f, acc[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+        for (int i0 = 0; i0 < a.C; i0 += CB) {
+            float kf[CB][EPL];
+#pragma unroll
+            for (int i = 0; i < CB; ++i) {
+                if (i0 + i < a.C) {
+                    load_f32<EPL>(children + (long long)(i0 + i) * a.child_stride + r * D + lane * EPL, kf[i]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) kf[i][e] = 0.f;
+                }
+            }
+            // lane i (< CB) fetches child i's bias for reference r
+            const float cb = lane < CB && i0 + lane < a.C
+                                 ? __ldg(children + (long long)(i0 + lane) * a.child_stride + a.child_bias + r)
+                                 : 0.f;
+            float part[CB];
+#pragma unroll
+            for (int i = 0; i < CB; ++i) {
+                float x = 0.f;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) x = fmaf(kf[i][e], q[e], x);
+                part[i] = x;
+            }
+            // lane group c = lane >> (5 - LG) ends with child c's dot product
+            const float dot = transpose_reduce<CB>(part, lane);
+            const int c = lane >> (5 - LG);
+            const float cbias = __shfl_sync(FULL, cb, c);  // every lane takes part in the shuffle
+            const float sc_own = i0 + c < a.C ? fmaf(a.beta, dot, cbias) : -INFINITY;
+            float s[CB];
+#pragma unroll
+            for (int i = 0; i < CB; ++i) s[i] = __shfl_sync(FULL, sc_own, i << (5 - LG));
+            float bm = m;
+#pragma unroll
+            for (int i = 0; i < CB; ++i) bm = fmaxf(bm, s[i]);
+            const float scale = expf(m - bm);
+            z *= scale;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] *= scale;
+#pragma unroll
+            for (int i = 0; i < CB; ++i) {
+                const float w = expf(s[i] - bm);
+                z += w;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, kf[i][e], acc[e]);
+            }
+            m = bm;
+        }
+        float *row = a.out + t * a.out_tree + j * a.NF + r * D + lane * EPL;
+        float x = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+            acc[e] = acc[e] / z;
+            x = fmaf(acc[e], q[e], x);
+        }
+        if constexpr (EPL % 4 == 0) {
+#pragma unroll
+            for (int e = 0; e < EPL; e += 4)
+                *reinterpret_cast<float4 *>(row + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+        } else {
+            *reinterpret_cast<float2 *>(row) = make_float2(acc[0], acc[1]);
+        }
+        const float dq = warp_sum(x);
+        if (lane == 0) a.out[t * a.out_tree + j * a.NF + (long long)a.R * D + r] = m + logf(z) - a.beta * dq;
+    }
+    chain_done();
+}
+
+// Blocks of the one-warp-per-item kernels: enough to give every warp several
+// items, at most 16 resident blocks' worth per SM.
+inline long long warp_blocks(long long warp_items) {
+    long long blocks = (warp_items + 31) / 32;
+    const long long cap = (long long)num_sms() * 16;
+    return blocks < 1 ? 1 : (blocks > cap ? cap : blocks);
+}
+
+template <typename KT, int D>
+cudaError_t launch_leaf(const zha_tree *t, const BuildArgs &a, cudaStream_t st) {
+    // RPW references per warp: RPW * D / 32 = 16 registers of references (at most R)
+    constexpr int RPW = 16 / (D / 32);
+    Probe pr(t, ZHA_K_BUILD, st);
+    if (a.R < RPW && a.R <= RPW / 2) {
+        if (a.R <= 1) return launch_chained(build_leaf_kernel<KT, D, 1>, dim3((unsigned)warp_blocks(a.items)),
+                                            dim3(256), 0, st, a);
+        if (a.R <= 2) return launch_chained(build_leaf_kernel<KT, D, (RPW >= 2 ? 2 : 1)>,
+                                            dim3((unsigned)warp_blocks(a.items)), dim3(256), 0, st, a);
+        if constexpr (RPW >= 8) {
+            if (a.R <= 4) return launch_chained(build_leaf_kernel<KT, D, 4>, dim3((unsigned)warp_blocks(a.items)),
+                                                dim3(256), 0, st, a);
+        }
+    }
+    const long long wpn = (a.R + RPW - 1) / RPW;
+    return launch_chained(build_leaf_kernel<KT, D, RPW>, dim3((unsigned)warp_blocks(a.items * wpn)), dim3(256), 0,
+                          st, a);
+}
+
+template <int D>
+cudaError_t launch_upper(const zha_tree *t, const BuildArgs &a, cudaStream_t st) {
+    Probe pr(t, ZHA_K_BUILD, st);
+    return launch_chained(build_upper_kernel<D>, dim3((unsigned)warp_blocks(a.items * a.R)), dim3(256), 0, st, a);
+}
+
 template <typename CT, int D>
 cudaError_t launch_build_typed(const zha_tree *t, const BuildArgs &a, cudaStream_t st) {
     const int threads = 32 * a.R;
@@ -179,6 +447,19 @@ cudaError_t launch_build_level(const zha_tree *t, int level, long long j0, long 
         a.child_bias = (long long)c.R * c.d;
     }
     const bool bf = keys && c.kv_dtype == ZHA_BF16;
+    if (!keys) {
+        switch (c.d) {
+            case 64: return launch_upper<64>(t, a, st);
+            case 128: return launch_upper<128>(t, a, st);
+            case 256: return launch_upper<256>(t, a, st);
+        }
+    } else {
+        switch (c.d) {
+            case 64: return bf ? launch_leaf<__nv_bfloat16, 64>(t, a, st) : launch_leaf<float, 64>(t, a, st);
+            case 128: return bf ? launch_leaf<__nv_bfloat16, 128>(t, a, st) : launch_leaf<float, 128>(t, a, st);
+            case 256: return bf ? launch_leaf<__nv_bfloat16, 256>(t, a, st) : launch_leaf<float, 256>(t, a, st);
+        }
+    }
     switch (c.d) {
         case 64:
             return bf ? launch_build_typed<__nv_bfloat16, 64>(t, a, st) : launch_build_typed<float, 64>(t, a, st);
