@@ -11,15 +11,15 @@
 //
 // Mapping (all arithmetic fp32; the softmax is taken online over batches of
 // children, so a node's children are read once):
-//   build_leaf_kernel   level 1: a warp per node and group of RPW references
-//                       (4 at D = 128: two warps per node at R = 8, the second
-//                       one's key reads hitting L1). Lane l owns D/32
-//                       consecutive columns of each key; the keys of a batch are
-//                       loaded together (all loads in flight at once), each key's
-//                       RPW dot products are summed across the warp by one
+//   build_leaf_kernel   level 1: a warp per node (a contiguous run of nodes per
+//                       warp), its references RPW at a time (4 at D = 128). Lane
+//                       l owns D/32 consecutive columns of each key; the node's
+//                       keys are loaded together (all loads in flight at once)
+//                       and kept for every reference group, each key's RPW dot
+//                       products are summed across the warp by one
 //                       transpose-reduce, and every lane then takes the weights
-//                       of its warp's references by shuffles to accumulate their
-//                       weighted keys in registers.
+//                       of the group's references by shuffles to accumulate
+//                       their weighted keys in registers.
 //   build_upper_kernel  levels >= 2: one warp per (node, reference), reading
 //                       row r of each child (consecutive warps take the rows of
 //                       one node, so the node is written row after row); the
@@ -129,49 +129,55 @@ __global__ void __launch_bounds__(512) build_nodes_kernel(BuildArgs a) {
     chain_done();
 }
 
-// Level-1 nodes: WPN = ceil(R / RPW) warps per node, each taking RPW of its
-// references (RPW a power of two; rows past R are zero and unused); the keys come
-// KB at a time (KB * D / 32 registers of keys per lane: 32, or 16 at D = 64).
-template <typename KT, int D, int RPW>
-__global__ void __launch_bounds__(256, 2) build_leaf_kernel(BuildArgs a) {
-    chain_start();
-    constexpr int EPL = D / 32;
-    constexpr int KB = 32 / EPL < 8 ? 32 / EPL : 8;  // keys per batch
-    constexpr int LG = ilog2(RPW);
-    const int lane = threadIdx.x & 31;
-    const int rr = lane >> (5 - LG);  // reference (of this warp's RPW) whose sums this lane ends with
-    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
-    const KT *K = static_cast<const KT *>(a.child);
-    const int wpn = (a.R + RPW - 1) / RPW;
-    const long long witems = a.items * wpn;
-
-    for (long long wi = gw; wi < witems; wi += nw) {
-        const long long item = wi / wpn;
-        const int r0 = (int)(wi - item * wpn) * RPW;
-        const long long t = item / a.per_tree;
-        const long long j = a.j0 + item % a.per_tree;
-        const int h = (int)(t % a.H_kv);
-        float q[RPW][EPL];
+// D/32 consecutive fp32 reference columns of one lane (16-byte or 8-byte loads,
+// through L1: every warp of a head reads the same rows).
+template <int EPL>
+__device__ __forceinline__ void load_ref(const float *p, float (&v)[EPL]) {
+    if constexpr (EPL == 2) {
+        const float2 x = __ldg(reinterpret_cast<const float2 *>(p));
+        v[0] = x.x;
+        v[1] = x.y;
+    } else {
 #pragma unroll
-        for (int r = 0; r < RPW; ++r) {
-            if (r0 + r < a.R) {
-                load_cached<EPL>(a.refs + ((long long)h * a.R + r0 + r) * D + lane * EPL, q[r]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) q[r][e] = 0.f;
-            }
+        for (int e = 0; e < EPL; e += 4) {
+            const float4 x = __ldg(reinterpret_cast<const float4 *>(p + e));
+            v[e] = x.x;
+            v[e + 1] = x.y;
+            v[e + 2] = x.z;
+            v[e + 3] = x.w;
         }
-        const KT *keys = K + t * a.child_tree + j * a.C * (long long)D + lane * EPL;
-        float m = -INFINITY, z = 0.f;  // running max and sum of exp, of reference r0 + rr
-        float acc[RPW][EPL];
-#pragma unroll
-        for (int r = 0; r < RPW; ++r)
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[r][e] = 0.f;
+    }
+}
 
-        for (int i0 = 0; i0 < a.C; i0 += KB) {
-            float kf[KB][EPL];
+// The summaries of references r0 .. r0 + RPW - 1 of one level-1 node (keys at
+// `keys`, this lane's columns). With have_keys the node's C <= KB keys are in kf
+// already; otherwise they are loaded KB at a time into kf and the softmax is
+// taken online over the batches.
+template <typename KT, int D, int RPW, int KB>
+__device__ __forceinline__ void leaf_group(const BuildArgs &a, const KT *keys, const float *refs_h, int r0,
+                                           float *node, int lane, float (&kf)[KB][D / 32], bool have_keys) {
+    constexpr int EPL = D / 32;
+    constexpr int LG = ilog2(RPW);
+    const int rr = lane >> (5 - LG);  // reference (of this group) whose sums this lane ends with
+    float q[RPW][EPL];
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+        if (r0 + r < a.R) {
+            load_ref<EPL>(refs_h + (long long)(r0 + r) * D + lane * EPL, q[r]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) q[r][e] = 0.f;
+        }
+    }
+    float m = -INFINITY, z = 0.f;  // running max and sum of exp, of reference r0 + rr
+    float acc[RPW][EPL];
+#pragma unroll
+    for (int r = 0; r < RPW; ++r)
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[r][e] = 0.f;
+
+    for (int i0 = 0; i0 < a.C; i0 += KB) {
+        if (!have_keys) {
 #pragma unroll
             for (int i = 0; i < KB; ++i) {
                 if (i0 + i < a.C) {
@@ -181,77 +187,125 @@ __global__ void __launch_bounds__(256, 2) build_leaf_kernel(BuildArgs a) {
                     for (int e = 0; e < EPL; ++e) kf[i][e] = 0.f;
                 }
             }
-            // s[i]: beta <k_i, q_rr> (lanes of reference rr)
-            float s[KB];
+        }
+        // s[i]: beta <k_i, q_rr> (lanes of reference rr)
+        float s[KB];
 #pragma unroll
-            for (int i = 0; i < KB; ++i) {
-                float part[RPW];
-#pragma unroll
-                for (int r = 0; r < RPW; ++r) {
-                    float x = 0.f;
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) x = fmaf(kf[i][e], q[r][e], x);
-                    part[r] = x;
-                }
-                const float dot = transpose_reduce<RPW>(part, lane);
-                s[i] = i0 + i < a.C ? a.beta * dot : -INFINITY;
-            }
-            float bm = m;
-#pragma unroll
-            for (int i = 0; i < KB; ++i) bm = fmaxf(bm, s[i]);
-            const float scale = expf(m - bm);  // 0 on the first batch (m = -inf)
-            z *= scale;
-            float wt[KB];
-#pragma unroll
-            for (int i = 0; i < KB; ++i) {
-                wt[i] = expf(s[i] - bm);
-                z += wt[i];
-            }
-            m = bm;
-            // every lane takes each reference's scale and weights from that
-            // reference's lanes and accumulates its columns of the RPW sums
+        for (int i = 0; i < KB; ++i) {
+            float part[RPW];
 #pragma unroll
             for (int r = 0; r < RPW; ++r) {
-                const int src = r << (5 - LG);
-                const float sc = __shfl_sync(FULL, scale, src);
+                float x = 0.f;
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) acc[r][e] *= sc;
-#pragma unroll
-                for (int i = 0; i < KB; ++i) {
-                    const float w = __shfl_sync(FULL, wt[i], src);
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) acc[r][e] = fmaf(w, kf[i][e], acc[r][e]);
-                }
+                for (int e = 0; e < EPL; ++e) x = fmaf(kf[i][e], q[r][e], x);
+                part[r] = x;
             }
+            const float dot = transpose_reduce<RPW>(part, lane);
+            s[i] = i0 + i < a.C ? a.beta * dot : -INFINITY;
         }
-        // key_r = acc_r / z_r; bias_r = m_r + log z_r - beta <key_r, q_r>
-        float *node = a.out + t * a.out_tree + j * a.NF;
-        float part[RPW];
+        float bm = m;
+#pragma unroll
+        for (int i = 0; i < KB; ++i) bm = fmaxf(bm, s[i]);
+        const float scale = expf(m - bm);  // 0 on the first batch (m = -inf)
+        z *= scale;
+        float wt[KB];
+#pragma unroll
+        for (int i = 0; i < KB; ++i) {
+            wt[i] = expf(s[i] - bm);
+            z += wt[i];
+        }
+        m = bm;
+        // every lane takes each reference's scale and weights from that
+        // reference's lanes and accumulates its columns of the RPW sums
 #pragma unroll
         for (int r = 0; r < RPW; ++r) {
-            const float zr = __shfl_sync(FULL, z, r << (5 - LG));
-            float x = 0.f;
+            const int src = r << (5 - LG);
+            const float sc = __shfl_sync(FULL, scale, src);
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) {
-                acc[r][e] = acc[r][e] / zr;
-                x = fmaf(acc[r][e], q[r][e], x);
-            }
-            part[r] = x;
-            if (r0 + r < a.R) {
-                float *row = node + (r0 + r) * D + lane * EPL;
-                if constexpr (EPL % 4 == 0) {
+            for (int e = 0; e < EPL; ++e) acc[r][e] *= sc;
 #pragma unroll
-                    for (int e = 0; e < EPL; e += 4)
-                        *reinterpret_cast<float4 *>(row + e) = make_float4(acc[r][e], acc[r][e + 1], acc[r][e + 2],
-                                                                           acc[r][e + 3]);
-                } else {
-                    *reinterpret_cast<float2 *>(row) = make_float2(acc[r][0], acc[r][1]);
-                }
+            for (int i = 0; i < KB; ++i) {
+                const float w = __shfl_sync(FULL, wt[i], src);
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) acc[r][e] = fmaf(w, kf[i][e], acc[r][e]);
             }
         }
-        const float dq = transpose_reduce<RPW>(part, lane);
-        if (r0 + rr < a.R && (lane & ((32 >> LG) - 1)) == 0)
-            node[a.R * D + r0 + rr] = m + logf(z) - a.beta * dq;
+    }
+    // key_r = acc_r / z_r; bias_r = m_r + log z_r - beta <key_r, q_r>
+    float part[RPW];
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+        const float inv = 1.f / __shfl_sync(FULL, z, r << (5 - LG));
+        float x = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+            acc[r][e] *= inv;
+            x = fmaf(acc[r][e], q[r][e], x);
+        }
+        part[r] = x;
+        if (r0 + r < a.R) {
+            float *row = node + (r0 + r) * D + lane * EPL;
+            if constexpr (EPL % 4 == 0) {
+#pragma unroll
+                for (int e = 0; e < EPL; e += 4)
+                    *reinterpret_cast<float4 *>(row + e) = make_float4(acc[r][e], acc[r][e + 1], acc[r][e + 2],
+                                                                       acc[r][e + 3]);
+            } else {
+                *reinterpret_cast<float2 *>(row) = make_float2(acc[r][0], acc[r][1]);
+            }
+        }
+    }
+    const float dq = transpose_reduce<RPW>(part, lane);
+    if (r0 + rr < a.R && (lane & ((32 >> LG) - 1)) == 0) node[a.R * D + r0 + rr] = m + logf(z) - a.beta * dq;
+}
+
+// Level-1 nodes, one warp per node: each warp takes a contiguous run of the
+// nodes (tree-major), and for each one the R references RPW at a time (RPW a
+// power of two; rows past R are zero and unused). A node of C <= KB keys loads
+// them once for all its reference groups (KB * D / 32 registers of keys per
+// lane: 32, or 16 at D = 64); larger chunks load them KB at a time per group.
+template <typename KT, int D, int RPW>
+__global__ void __launch_bounds__(256, 2) build_leaf_kernel(BuildArgs a) {
+    chain_start();
+    constexpr int EPL = D / 32;
+    constexpr int KB = 32 / EPL < 8 ? 32 / EPL : 8;  // keys per batch
+    const int lane = threadIdx.x & 31;
+    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+    const KT *K = static_cast<const KT *>(a.child);
+    const long long per_warp = (a.items + nw - 1) / nw;
+    long long item = gw * per_warp;
+    const long long item_end = item + per_warp < a.items ? item + per_warp : a.items;
+    if (item < item_end) {
+        long long t = item / a.per_tree;
+        long long jj = item - t * a.per_tree;  // node of tree t, counted from j0
+        int h = (int)(t % a.H_kv);
+        const bool have_keys = a.C <= KB;
+        for (; item < item_end; ++item) {
+            const long long j = a.j0 + jj;
+            const KT *keys = K + t * a.child_tree + j * a.C * (long long)D + lane * EPL;
+            const float *refs_h = a.refs + (long long)h * a.R * D;
+            float *node = a.out + t * a.out_tree + j * a.NF;
+            float kf[KB][EPL];
+            if (have_keys) {
+#pragma unroll
+                for (int i = 0; i < KB; ++i) {
+                    if (i < a.C) {
+                        load_cached<EPL>(keys + (long long)i * D, kf[i]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < EPL; ++e) kf[i][e] = 0.f;
+                    }
+                }
+            }
+            for (int r0 = 0; r0 < a.R; r0 += RPW)
+                leaf_group<KT, D, RPW, KB>(a, keys, refs_h, r0, node, lane, kf, have_keys);
+            if (++jj == a.per_tree) {
+                jj = 0;
+                ++t;
+                h = h + 1 == a.H_kv ? 0 : h + 1;
+            }
+        }
     }
     chain_done();
 }
@@ -259,7 +313,7 @@ __global__ void __launch_bounds__(256, 2) build_leaf_kernel(BuildArgs a) {
 // Levels >= 2, one warp per (node, reference r): row r of each child, CB at a
 // time (CB * D / 32 registers of rows per lane).
 template <int D>
-__global__ void __launch_bounds__(256, 2) build_upper_kernel(BuildArgs a) {
+__global__ void __launch_bounds__(256, 3) build_upper_kernel(BuildArgs a) {
     chain_start();
     constexpr int EPL = D / 32;
     constexpr int CB = 32 / EPL;  // children per batch
@@ -269,15 +323,23 @@ __global__ void __launch_bounds__(256, 2) build_upper_kernel(BuildArgs a) {
     const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
     const float *nodes = static_cast<const float *>(a.child);
     const long long witems = a.items * a.R;
-
-    for (long long wi = gw; wi < witems; wi += nw) {
-        const long long item = wi / a.R;
-        const int r = (int)(wi - item * a.R);
-        const long long t = item / a.per_tree;
-        const long long j = a.j0 + item % a.per_tree;
-        const int h = (int)(t % a.H_kv);
+    // a contiguous run of (node, reference) pairs per warp, indices advanced in step
+    const long long per_warp = (witems + nw - 1) / nw;
+    long long wi = gw * per_warp;
+    const long long wi_end = wi + per_warp < witems ? wi + per_warp : witems;
+    if (wi >= wi_end) {
+        chain_done();
+        return;
+    }
+    long long item = wi / a.R;
+    int r = (int)(wi - item * a.R);
+    long long t = item / a.per_tree;
+    long long jj = item - t * a.per_tree;
+    int h = (int)(t % a.H_kv);
+    for (; wi < wi_end; ++wi) {
+        const long long j = a.j0 + jj;
         float q[EPL];
-        load_cached<EPL>(a.refs + ((long long)h * a.R + r) * D + lane * EPL, q);
+        load_ref<EPL>(a.refs + ((long long)h * a.R + r) * D + lane * EPL, q);
         const float *children = nodes + t * a.child_tree + j * a.C * a.child_stride;
         float m = -INFINITY, z = 0.f, acc[EPL];
 #pragma unroll
@@ -330,10 +392,11 @@ __global__ void __launch_bounds__(256, 2) build_upper_kernel(BuildArgs a) {
             m = bm;
         }
         float *row = a.out + t * a.out_tree + j * a.NF + r * D + lane * EPL;
+        const float inv = 1.f / z;
         float x = 0.f;
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
-            acc[e] = acc[e] / z;
+            acc[e] *= inv;
             x = fmaf(acc[e], q[e], x);
         }
         if constexpr (EPL % 4 == 0) {
@@ -345,6 +408,14 @@ __global__ void __launch_bounds__(256, 2) build_upper_kernel(BuildArgs a) {
         }
         const float dq = warp_sum(x);
         if (lane == 0) a.out[t * a.out_tree + j * a.NF + (long long)a.R * D + r] = m + logf(z) - a.beta * dq;
+        if (++r == a.R) {
+            r = 0;
+            if (++jj == a.per_tree) {
+                jj = 0;
+                ++t;
+                h = h + 1 == a.H_kv ? 0 : h + 1;
+            }
+        }
     }
     chain_done();
 }
@@ -359,22 +430,16 @@ inline long long warp_blocks(long long warp_items) {
 
 template <typename KT, int D>
 cudaError_t launch_leaf(const zha_tree *t, const BuildArgs &a, cudaStream_t st) {
-    // RPW references per warp: RPW * D / 32 = 16 registers of references (at most R)
+    // RPW references at a time: RPW * D / 32 = 16 registers of references (fewer when R is small)
     constexpr int RPW = 16 / (D / 32);
+    const dim3 grid((unsigned)warp_blocks(a.items));
     Probe pr(t, ZHA_K_BUILD, st);
-    if (a.R < RPW && a.R <= RPW / 2) {
-        if (a.R <= 1) return launch_chained(build_leaf_kernel<KT, D, 1>, dim3((unsigned)warp_blocks(a.items)),
-                                            dim3(256), 0, st, a);
-        if (a.R <= 2) return launch_chained(build_leaf_kernel<KT, D, (RPW >= 2 ? 2 : 1)>,
-                                            dim3((unsigned)warp_blocks(a.items)), dim3(256), 0, st, a);
-        if constexpr (RPW >= 8) {
-            if (a.R <= 4) return launch_chained(build_leaf_kernel<KT, D, 4>, dim3((unsigned)warp_blocks(a.items)),
-                                                dim3(256), 0, st, a);
-        }
+    if (a.R <= 1) return launch_chained(build_leaf_kernel<KT, D, 1>, grid, dim3(256), 0, st, a);
+    if (a.R <= 2 && RPW >= 4) return launch_chained(build_leaf_kernel<KT, D, 2>, grid, dim3(256), 0, st, a);
+    if constexpr (RPW >= 8) {
+        if (a.R <= 4) return launch_chained(build_leaf_kernel<KT, D, 4>, grid, dim3(256), 0, st, a);
     }
-    const long long wpn = (a.R + RPW - 1) / RPW;
-    return launch_chained(build_leaf_kernel<KT, D, RPW>, dim3((unsigned)warp_blocks(a.items * wpn)), dim3(256), 0,
-                          st, a);
+    return launch_chained(build_leaf_kernel<KT, D, RPW>, grid, dim3(256), 0, st, a);
 }
 
 template <int D>
