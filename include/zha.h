@@ -266,6 +266,83 @@ int zha_chunk_mass(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_hea
 int zha_ref_grad(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q, float *loss, float *grad,
                  void *stream);
 
+/* ---------------------------------------------------------------------------
+ * Context-parallel walk. [P4] abstract: the method aims at contexts of
+ * hundreds of millions of tokens, more than one GPU holds. The keys of each
+ * tree are then split across processes in runs of whole top-level nodes
+ * (C^depth keys each; the last process also holds the keys past the last full
+ * top node, so it has the orphans and the tail). Each process builds its shard
+ * with zha_build over its keys (fixed depth): because the runs align with the
+ * top nodes, the shard's level-l nodes are, bit for bit, the nodes
+ * key_begin / C^l onward of the tree over all keys. The walk of zha_search
+ * ([P1] "Run a small tree yourself", route; "How does top-p differ from top-K?")
+ * is then taken one level at a time, with an exchange between the steps that
+ * the caller makes over its process group (an all-gather, in process order):
+ *   zha_cp_begin   once: queries, the start level (from the whole tree's
+ *                  counts) and this shard's start frontier;
+ *   zha_cp_export  per level: score this shard's frontier and write each
+ *                  walk's (global node id, score) list, ids ascending;
+ *   zha_cp_select  per level, after the all-gather: choose over the gathered
+ *                  lists exactly as zha_search chooses over the whole frontier
+ *                  (same selector, same order, so the same nodes), keep the
+ *                  opened nodes this shard holds, and make its next frontier;
+ *                  at level 1 write this shard's chosen chunks and end.
+ * Every process makes the same sequence of calls and exchanges. The final
+ * attention ([P1] "Common misunderstandings": ordinary attention over the
+ * chosen original keys) is zha_attend on each shard (its chosen chunks, and on
+ * the last process the tail), merged across processes by zha_lse_combine.
+ */
+
+/*
+ * zha_cp_begin: start a context-parallel walk of Q on this shard.
+ * key_begin: index of the shard's first key in the whole sequence, a multiple
+ *   of C^depth; global_counts[0..depth] (host): keys and nodes per level of
+ *   the tree over all keys (the sum of the shards' counts); n_counts = depth + 1.
+ * *start_level receives the level the walk starts at (the lowest holding at
+ *   most top_width nodes in the whole tree, else depth).
+ * Errors: ZHA_ERR_INVALID (a growing tree, misaligned key_begin, counts below
+ * this shard's), ZHA_ERR_OOM, ZHA_ERR_CUDA.
+ */
+int zha_cp_begin(zha_tree *tree, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q, long long key_begin,
+                 const long long *global_counts, int n_counts, int *start_level, void *stream);
+
+/*
+ * zha_cp_export: score this shard's frontier at the current level and write,
+ * per walk w, counts[w] pairs ids[w][i] (global node id, ascending) and
+ * scores[w][i] (max over r of beta*<key_r, q> + bias_r), rows of list_stride.
+ * A frontier longer than list_stride keeps its first list_stride entries and
+ * makes zha_sync_status return ZHA_ERR_CAPACITY (the shard's level-1 node count
+ * always suffices). *level receives the level exported.
+ */
+int zha_cp_export(zha_tree *tree, int *ids, float *scores, int *counts, long long list_stride, int *level,
+                  void *stream);
+
+/*
+ * zha_cp_select: the choice at the current level over the whole frontier.
+ * ids, scores: [n_parts][walks][list_stride], counts: [n_parts][walks] (device),
+ *   the exports of every process in process order (the all-gather of
+ *   zha_cp_export's outputs).
+ * mode, p, k: as zha_search. At level 1, sel [walks][max_sel] and sel_count
+ *   receive this shard's chosen chunks (local level-1 ids: chunk c covers the
+ *   shard's keys C*c .. C*c+C-1), as zha_search writes them for a whole tree.
+ * *level receives the next level to export, or 0 when the walk is complete.
+ * Scratch of about 16 * walks * n_parts * list_stride bytes is taken from the
+ * tree's second scratch block (grown when too small).
+ */
+int zha_cp_select(zha_tree *tree, int n_parts, const int *ids, const float *scores, const int *counts,
+                  long long list_stride, zha_mode mode, float p, int k, int *sel, int *sel_count, int max_sel,
+                  int *level, void *stream);
+
+/*
+ * zha_lse_combine: attention over the union of disjoint key sets from the
+ * attentions over each: outs [n_parts][walks][d] fp32 and lses [n_parts][walks]
+ * (each part's out and lse, as zha_attend returns them; lse = -inf for a part
+ * without keys) give out = sum_p exp(lse_p - lse) out_p and lse = logsumexp_p
+ * lse_p. out: [walks][d] of out_dtype; lse: [walks] fp32 or NULL. No tree.
+ */
+int zha_lse_combine(int n_parts, long long walks, int d, const float *outs, const float *lses, void *out,
+                    zha_dtype out_dtype, float *lse, void *stream);
+
 /*
  * zha_reserve: allocate the search and attend scratch for up to max_walks walks
  * and selections of up to max_sel chunks now, so that later calls with at most

@@ -74,6 +74,8 @@ def test_host_side_argument_checks(zha):
     assert L.zha_append(None, None, None, None) == zha.ERR_INVALID
     assert L.zha_rebuild(None, None) == zha.ERR_INVALID
     assert L.zha_test_wait_limit(None, 1000, 1) == zha.ERR_INVALID
+    assert L.zha_cp_export(None, None, None, None, 1, None, None) == zha.ERR_INVALID
+    assert L.zha_lse_combine(0, 1, 64, None, None, None, 0, None, None) == zha.ERR_INVALID
     assert L.zha_reserve(None, 1, 1) == zha.ERR_INVALID
     assert L.zha_dense_scan(None, None, 0, 1, 1, 0, 0.9, 1, None, None, 1, None) == zha.ERR_INVALID
     assert L.zha_chunk_mass(None, None, 0, 1, 1, 16, 0.9, None, None, 1, None) == zha.ERR_INVALID

@@ -29,7 +29,7 @@ SYMBOLS = ("zha_build", "zha_append", "zha_search", "zha_attend", "zha_reserve",
            "zha_num_keys", "zha_depth", "zha_sync_status", "zha_destroy", "zha_last_error", "zha_version",
            "zha_profile", "zha_profile_read", "zha_kernel_launches", "zha_last_search_info",
            "zha_dense_scan", "zha_attend_noalloc", "zha_chunk_mass", "zha_ref_grad", "zha_rebuild",
-           "zha_test_wait_limit")
+           "zha_test_wait_limit", "zha_cp_begin", "zha_cp_export", "zha_cp_select", "zha_lse_combine")
 KERNEL_KINDS = ("build", "append", "search_init", "score", "select", "attend_plan", "attend_partial",
                 "attend_combine", "score_tc")
 
@@ -79,6 +79,10 @@ def lib():
         L.zha_append.argtypes = [vp, vp, vp, vp]
         L.zha_rebuild.argtypes = [vp, vp]
         L.zha_test_wait_limit.argtypes = [vp, ll, i]
+        L.zha_cp_begin.argtypes = [vp, vp, i, i, i, ll, ctypes.POINTER(ll), i, ctypes.POINTER(i), vp]
+        L.zha_cp_export.argtypes = [vp, vp, vp, vp, ll, ctypes.POINTER(i), vp]
+        L.zha_cp_select.argtypes = [vp, i, vp, vp, vp, ll, i, f, i, vp, vp, i, ctypes.POINTER(i), vp]
+        L.zha_lse_combine.argtypes = [i, ll, i, vp, vp, vp, i, vp, vp]
         L.zha_search.argtypes = [vp, vp, i, i, i, i, f, i, vp, vp, i, vp, vp]
         L.zha_attend.argtypes = [vp, vp, i, i, i, vp, vp, i, vp, i, vp, vp]
         L.zha_attend_noalloc.argtypes = [vp, vp, i, i, i, vp, vp, i, vp, i, vp, vp]
@@ -306,6 +310,34 @@ class Tree:
                                   _dev(grad, "grad"), _stream(stream)))
         return loss, grad
 
+    # -- context-parallel walk (one shard of every tree per process) ------------
+    def cp_begin(self, Q: torch.Tensor, key_begin: int, global_counts, stream=None) -> int:
+        """Start a context-parallel walk of Q on this shard; returns the start level."""
+        B, Hq, nq, d = Q.shape
+        counts = (ctypes.c_longlong * len(global_counts))(*[int(c) for c in global_counts])
+        level = ctypes.c_int()
+        _check(lib().zha_cp_begin(self._h, _dev(Q, "Q"), _dtype_code(Q), Hq, nq, int(key_begin), counts,
+                                  len(global_counts), ctypes.byref(level), _stream(stream)))
+        return level.value
+
+    def cp_export(self, ids: torch.Tensor, scores: torch.Tensor, counts: torch.Tensor, stream=None) -> int:
+        """Score this shard's frontier; ids/scores [walks][stride], counts [walks]. Returns the level."""
+        level = ctypes.c_int()
+        _check(lib().zha_cp_export(self._h, _dev(ids, "ids"), _dev(scores, "scores"), _dev(counts, "counts"),
+                                   ids.shape[1], ctypes.byref(level), _stream(stream)))
+        return level.value
+
+    def cp_select(self, ids: torch.Tensor, scores: torch.Tensor, counts: torch.Tensor, mode: int, p: float, k: int,
+                  sel: torch.Tensor, sel_count: torch.Tensor, stream=None) -> int:
+        """Choose over the gathered lists (ids/scores [parts][walks][stride], counts
+        [parts][walks]); returns the next level (0 when the walk is complete)."""
+        level = ctypes.c_int()
+        _check(lib().zha_cp_select(self._h, ids.shape[0], _dev(ids, "ids"), _dev(scores, "scores"),
+                                   _dev(counts, "counts"), ids.shape[2], mode, float(p), int(k), _dev(sel, "sel"),
+                                   _dev(sel_count, "sel_count"), sel.shape[1], ctypes.byref(level),
+                                   _stream(stream)))
+        return level.value
+
     def reserve(self, max_walks: int, max_sel: int) -> None:
         _check(lib().zha_reserve(self._h, int(max_walks), int(max_sel)))
 
@@ -343,6 +375,17 @@ class Tree:
             self.close()
         except Exception:
             pass
+
+
+def lse_combine(outs: torch.Tensor, lses: torch.Tensor, out_dtype=torch.float32, stream=None):
+    """Attention over the union of disjoint key sets: outs [parts][walks][d] fp32,
+    lses [parts][walks] fp32 -> (out [walks][d] of out_dtype, lse [walks])."""
+    P, W, d = outs.shape
+    out = torch.empty(W, d, dtype=out_dtype, device=outs.device)
+    lse = torch.empty(W, dtype=torch.float32, device=outs.device)
+    _check(lib().zha_lse_combine(P, W, d, _dev(outs, "outs"), _dev(lses, "lses"), _dev(out, "out"),
+                                 _dtype_code(out), _dev(lse, "lse"), _stream(stream)))
+    return out, lse
 
 
 def parse_stats(st: torch.Tensor) -> list:

@@ -378,6 +378,125 @@ int zha_search(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads, int
     return ZHA_OK;
 }
 
+int zha_cp_begin(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q, long long key_begin,
+                 const long long *global_counts, int n_counts, int *start_level, void *stream) {
+    long long W;
+    int G;
+    int rc = check_queries(t, Q, q_dtype, n_q_heads, n_q, &W, &G);
+    if (rc) return rc;
+    if (!global_counts || !start_level) return fail(ZHA_ERR_INVALID, "global_counts and start_level must not be NULL");
+    if (t->grow) return fail(ZHA_ERR_INVALID, "the context-parallel walk needs a tree of fixed depth");
+    const int depth = t->cfg.depth, C = t->cfg.chunk;
+    if (n_counts != depth + 1) return fail(ZHA_ERR_INVALID, "global_counts must hold depth + 1 = %d counts", depth + 1);
+    long long span = 1;
+    for (int l = 0; l < depth; ++l) span *= C;
+    if (key_begin < 0 || key_begin % span)
+        return fail(ZHA_ERR_INVALID, "key_begin must be a multiple of C^depth = %lld", span);
+    long long div = 1;
+    for (int l = 0; l <= depth; ++l) {
+        const long long off = key_begin / div;
+        const long long mine = l == 0 ? t->n : t->n_nodes[l];
+        if (global_counts[l] < off + mine)
+            return fail(ZHA_ERR_INVALID, "global count of level %d (%lld) is below this shard's end (%lld)", l,
+                        global_counts[l], off + mine);
+        t->cp_off[l] = off;
+        div *= C;
+    }
+    int s0 = depth;
+    for (int l = 1; l <= depth; ++l)
+        if (global_counts[l] <= t->cfg.top_width) {
+            s0 = l;
+            break;
+        }
+    zha::Scratch s;
+    rc = zha::reserve(t, W, 1, &s);
+    if (rc) return rc;
+    ZHA_CUDA(zha::launch_search_init(t, s, Q, q_dtype, G, W, nullptr, s0, static_cast<cudaStream_t>(stream)),
+             "launching the walk set-up");
+    t->cp_active = 1;
+    t->cp_level = s0;
+    t->cp_start = s0;
+    t->cp_cur = 0;
+    t->cp_W = W;
+    t->cp_G = G;
+    *start_level = s0;
+    return ZHA_OK;
+}
+
+int zha_cp_export(zha_tree *t, int *ids, float *scores, int *counts, long long list_stride, int *level,
+                  void *stream) {
+    if (!t || !ids || !scores || !counts || !level) return fail(ZHA_ERR_INVALID, "NULL argument");
+    if (!t->cp_active) return fail(ZHA_ERR_INVALID, "no context-parallel walk is in progress (zha_cp_begin)");
+    if (list_stride < 1) return fail(ZHA_ERR_INVALID, "list_stride must be >= 1");
+    zha::Scratch s;
+    int rc = zha::reserve(t, t->cp_W, 1, &s);
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int l = t->cp_level;
+    ZHA_CUDA(zha::launch_score_level(t, s, l, t->cp_G, st), "launching the shard's scoring");
+    ZHA_CUDA(zha::launch_cp_export(t, s, t->cp_cur, l, l == t->cp_start, t->cp_off[l], t->cp_W, ids, scores, counts,
+                                   list_stride, st),
+             "launching the frontier export");
+    *level = l;
+    return ZHA_OK;
+}
+
+int zha_cp_select(zha_tree *t, int n_parts, const int *ids, const float *scores, const int *counts,
+                  long long list_stride, zha_mode mode, float p, int k, int *sel, int *sel_count, int max_sel,
+                  int *level, void *stream) {
+    if (!t || !ids || !scores || !counts || !sel || !sel_count || !level) return fail(ZHA_ERR_INVALID, "NULL argument");
+    if (!t->cp_active) return fail(ZHA_ERR_INVALID, "no context-parallel walk is in progress (zha_cp_begin)");
+    if (n_parts < 1 || list_stride < 1 || max_sel < 1)
+        return fail(ZHA_ERR_INVALID, "n_parts, list_stride and max_sel must be >= 1");
+    if (mode == ZHA_TOP_P) {
+        if (!(p > 0.f) || std::isnan(p)) return fail(ZHA_ERR_INVALID, "top-p needs p > 0 (got %g)", (double)p);
+    } else if (mode == ZHA_TOP_K) {
+        if (k < 1) return fail(ZHA_ERR_INVALID, "top-K needs k >= 1 (got %d)", k);
+    } else {
+        return fail(ZHA_ERR_INVALID, "mode must be ZHA_TOP_P or ZHA_TOP_K");
+    }
+    const long long W = t->cp_W, P = (long long)n_parts * list_stride;
+    if (P > (1LL << 30)) return fail(ZHA_ERR_INVALID, "n_parts * list_stride too large");
+    zha::Scratch s;
+    int rc = zha::reserve(t, W, 1, &s);
+    if (rc) return rc;
+    // packed lists, chosen ids and the selector's staging, per walk P slots each
+    const size_t o_ps = align_up(sizeof(int) * W * P), o_pc = o_ps + align_up(sizeof(float) * W * P);
+    const size_t o_op = o_pc + align_up(sizeof(int) * W), o_oc = o_op + align_up(sizeof(int) * W * P);
+    const size_t o_st = o_oc + align_up(sizeof(int) * W);
+    rc = zha::grow_dense_scratch(t, o_st + align_up(sizeof(uint32_t) * W * P));
+    if (rc) return rc;
+    char *b = static_cast<char *>(t->dws);
+    zha::CpScratch cs{reinterpret_cast<int *>(b), reinterpret_cast<float *>(b + o_ps), reinterpret_cast<int *>(b + o_pc),
+                      reinterpret_cast<int *>(b + o_op), reinterpret_cast<int *>(b + o_oc),
+                      reinterpret_cast<uint32_t *>(b + o_st), P};
+    const int l = t->cp_level;
+    ZHA_CUDA(zha::launch_cp_select(t, s, t->cp_cur, l, t->cp_G, W, n_parts, ids, scores, counts, list_stride, mode, p,
+                                   k, cs, t->cp_off[l], sel, sel_count, max_sel, static_cast<cudaStream_t>(stream)),
+             "launching the context-parallel choice");
+    if (l == 1) {
+        t->cp_active = 0;
+        *level = 0;
+    } else {
+        t->cp_cur ^= 1;
+        t->cp_level = l - 1;
+        *level = l - 1;
+    }
+    return ZHA_OK;
+}
+
+int zha_lse_combine(int n_parts, long long walks, int d, const float *outs, const float *lses, void *out,
+                    zha_dtype out_dtype, float *lse, void *stream) {
+    if (n_parts < 1 || walks < 1 || d < 1) return fail(ZHA_ERR_INVALID, "n_parts, walks and d must be >= 1");
+    if (!outs || !lses || !out) return fail(ZHA_ERR_INVALID, "outs, lses and out must not be NULL");
+    if (out_dtype != ZHA_F32 && out_dtype != ZHA_BF16) return fail(ZHA_ERR_INVALID, "out_dtype must be ZHA_F32 or ZHA_BF16");
+    if (walks > (1LL << 31) - 1) return fail(ZHA_ERR_INVALID, "too many walks");
+    ZHA_CUDA(zha::launch_lse_combine(n_parts, walks, d, outs, lses, out, out_dtype, lse,
+                                     static_cast<cudaStream_t>(stream)),
+             "launching the log-sum-exp combine");
+    return ZHA_OK;
+}
+
 int zha_attend(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads, int n_q, const int *sel,
                const int *sel_count, int max_sel, void *out, zha_dtype out_dtype, float *lse, void *stream) {
     long long W;
@@ -390,6 +509,16 @@ int zha_attend(zha_tree *t, const void *Q, zha_dtype q_dtype, int n_q_heads, int
     zha::Scratch s;
     rc = zha::reserve(t, W, max_sel, &s);
     if (rc) return rc;
+    if (t->cfg.d == 128 && zha::attend_tc_applicable(t, G, q_dtype)) {
+        // many bf16 walks per tree: tree-major attention on the tensor cores, its
+        // scratch from the tree's second block
+        rc = zha::grow_dense_scratch(t, zha::attend_tc_scratch(t, G, W));
+        if (rc) return rc;
+        ZHA_CUDA(zha::launch_attend_tc(t, G, W, Q, sel, sel_count, max_sel, out, out_dtype, lse, t->dws,
+                                       static_cast<cudaStream_t>(stream)),
+                 "launching the tensor-core attention");
+        return ZHA_OK;
+    }
     ZHA_CUDA(zha::launch_attend(t, s, Q, q_dtype, G, W, sel, sel_count, max_sel, out, out_dtype, lse,
                                 static_cast<cudaStream_t>(stream)),
              "launching the attention");

@@ -200,6 +200,11 @@ struct zha_tree {
     struct zha_profiler *prof;  // NULL unless zha_profile(tree, 1)
     unsigned long long tc_wait_ns;  // limit of the tensor-core scorer's waits (0: 1 s)
     int tc_stall;                   // test hook of zha_test_wait_limit
+
+    // context-parallel walk (zha_cp_begin / zha_cp_export / zha_cp_select)
+    int cp_active, cp_level, cp_start, cp_cur, cp_G;
+    long long cp_W;
+    long long cp_off[ZHA_MAX_DEPTH + 1];  // global id of the shard's first node, per level
     long long last_W;
     int last_G, last_start, last_max_sel;
 };
@@ -232,6 +237,18 @@ struct Scratch {
 };
 
 int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s);
+
+// Packed lists of a context-parallel level step (carved from the tree's second
+// scratch block): per walk P = n_parts * list stride slots.
+struct CpScratch {
+    int *pids;
+    float *pscores;
+    int *pcount;
+    int *opened;
+    int *ocount;
+    uint32_t *stage;
+    long long P;
+};
 
 // Byte offsets of the attention's scratch for W walks of head dimension D, in
 // one block of `bytes` (offsets 256-byte aligned); its size depends on W and D only.
@@ -279,6 +296,24 @@ cudaError_t launch_append_kv(const zha_tree *t, const void *k_new, const void *v
 cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zha_dtype q_dtype,
                           int G, long long W, int mode, float p, int k, int *sel, int *sel_count,
                           int max_sel, zha_stats *stats, int start_level, cudaStream_t st);
+cudaError_t launch_search_init(const zha_tree *t, const Scratch &s, const void *Q, zha_dtype q_dtype, int G,
+                               long long W, zha_stats *stats, int start_level, cudaStream_t st);
+cudaError_t launch_score_level(const zha_tree *t, const Scratch &s, int l, int G, cudaStream_t st);
+cudaError_t launch_cp_export(const zha_tree *t, const Scratch &s, int cur, int level, bool start, long long off,
+                             long long W, int *ids, float *scores, int *counts, long long stride, cudaStream_t st);
+cudaError_t launch_cp_select(const zha_tree *t, const Scratch &s, int cur, int level, int G, long long W, int n_parts,
+                             const int *ids, const float *scores, const int *counts, long long stride, int mode,
+                             float p, int k, const CpScratch &cs, long long lo, int *sel, int *sel_count,
+                             int max_sel, cudaStream_t st);
+cudaError_t launch_lse_combine(int n_parts, long long W, int D, const float *outs, const float *lses, void *out,
+                               zha_dtype out_dtype, float *lse, cudaStream_t st);
+// Final attention on the tensor cores for trees walked by many bf16 queries
+// (zha_attend_tc.cu): applicability, scratch bytes, and the launch (scratch at ws).
+bool attend_tc_applicable(const zha_tree *t, int G, zha_dtype q_dtype);
+size_t attend_tc_scratch(const zha_tree *t, int G, long long W);
+cudaError_t launch_attend_tc(const zha_tree *t, int G, long long W, const void *Q, const int *sel,
+                             const int *sel_count, int max_sel, void *out, zha_dtype out_dtype, float *lse,
+                             void *ws, cudaStream_t st);
 cudaError_t launch_attend(const zha_tree *t, const Scratch &s, const void *Q, zha_dtype q_dtype,
                           int G, long long W, const int *sel, const int *sel_count, int max_sel,
                           void *out, zha_dtype out_dtype, float *lse, cudaStream_t st);

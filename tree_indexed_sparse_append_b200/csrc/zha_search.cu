@@ -356,11 +356,20 @@ struct SelectArgs {
     int *status;
     long long smem_keys;     // frontiers up to this size are staged in shared memory
     uint32_t *gkey;          // [W][Sstride] staging for larger frontiers
+    // explicit frontiers (the context-parallel walk): per walk, list_count[w]
+    // (node id, score) pairs at list_ids / list_scores + w * list_stride, ids
+    // ascending; S, par_in and the orphan counts are then unused
+    const int *list_ids;
+    const float *list_scores;
+    const int *list_count;
+    long long list_stride;
 };
 
-// frontier position -> node id (positions and ids fit in 32 bits)
-__device__ __forceinline__ long long frontier_id(const SelectArgs &a, const int *par, long long npar,
+// frontier position -> node id (positions and ids fit in 32 bits); lid: the
+// walk's explicit list, if any
+__device__ __forceinline__ long long frontier_id(const SelectArgs &a, const int *lid, const int *par, long long npar,
                                                  long long i) {
+    if (lid) return lid[i];
     if (a.start) return i;
     const int ii = (int)i, C = a.C;
     const int kids = (int)npar * C;
@@ -446,9 +455,11 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
     const long long walk = blockIdx.x;
     const int tid = threadIdx.x;
     const int t = (int)(walk / a.G), g = (int)(walk % a.G);
-    const long long npar = a.start ? 0 : a.n_par_in[walk];
-    const int *par = a.par_in + walk * a.Lstride;
-    const long long F = a.start ? a.n_level : npar * a.C + a.n_orph;
+    const int *lid = a.list_ids ? a.list_ids + walk * a.list_stride : nullptr;
+    const float *lsc = a.list_scores ? a.list_scores + walk * a.list_stride : nullptr;
+    const long long npar = a.start || lid ? 0 : a.n_par_in[walk];
+    const int *par = lid ? nullptr : a.par_in + walk * a.Lstride;
+    const long long F = lid ? a.list_count[walk] : (a.start ? a.n_level : npar * a.C + a.n_orph);
     const float *S = a.S + walk * a.Sstride;
     uint32_t *skey = F <= a.smem_keys ? skey_s : a.gkey + walk * a.Sstride;
     auto key_at = [&](long long i) -> uint32_t { return skey[i]; };
@@ -460,10 +471,10 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
     for (long long i = tid; i < F; i += 8 * NT) {
         long long id[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) id[u] = i + u * NT < F ? frontier_id(a, par, npar, i + u * NT) : -1;
+        for (int u = 0; u < 8; ++u) id[u] = i + u * NT < F ? frontier_id(a, lid, par, npar, i + u * NT) : -1;
         float v[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = id[u] >= 0 ? S[id[u]] : 0.f;
+        for (int u = 0; u < 8; ++u) v[u] = id[u] >= 0 ? (lsc ? lsc[i + u * NT] : S[id[u]]) : 0.f;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             if (id[u] >= 0) {
@@ -690,7 +701,7 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const long long i = i00 + 32 * u + lane;
-                idv[u] = i < rend ? frontier_id(a, par, npar, i) : 0;
+                idv[u] = i < rend ? frontier_id(a, lid, par, npar, i) : 0;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -706,7 +717,7 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
                         if (r < (unsigned)a.max_sel) a.sel[walk * a.max_sel + r] = (int)id;
                     } else {
                         a.par_out[walk * a.Lstride + r] = (int)id;
-                        set_bits(M_tree, U_tree, a.G, g, id * a.C, id * a.C + a.C);
+                        if (M_tree) set_bits(M_tree, U_tree, a.G, g, id * a.C, id * a.C + a.C);
                     }
                 }
                 rank += __popc(om);
@@ -838,18 +849,13 @@ cudaError_t launch_select_all(const zha_tree *t, const float *S, uint32_t *gkey,
     return launch_select<256>(se, W, st);
 }
 
-cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zha_dtype q_dtype, int G,
-                          long long W, int mode, float p, int k, int *sel, int *sel_count, int max_sel,
-                          zha_stats *stats, int start_level, cudaStream_t st) {
-    const zha_config &c = t->cfg;
-    const int D = c.d, C = c.chunk;
-    cudaError_t e;
+cudaError_t launch_search_init(const zha_tree *t, const Scratch &s, const void *Q, zha_dtype q_dtype, int G,
+                               long long W, zha_stats *stats, int start_level, cudaStream_t st) {
     auto words = [&](int l) { return (t->cap_nodes[l] + 31) / 32; };
-
     InitArgs ia{};
     ia.Q = Q;
     ia.q_bf16 = q_dtype == ZHA_BF16;
-    ia.D = D;
+    ia.D = t->cfg.d;
     ia.W = W;
     ia.qf = s.qf;
     ia.n_par = s.cnt[0];
@@ -864,10 +870,43 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
     ia.U_all = s.U_base;
     ia.M_all_words = (long long)(s.M_bytes / sizeof(unsigned));
     ia.U_all_words = (long long)(s.U_bytes / sizeof(unsigned));
-    {
-        Probe pr(t, ZHA_K_SEARCH_INIT, st);
-        if ((e = launch_chained(search_init_kernel, dim3((unsigned)W), dim3(128), 0, st, ia)) != cudaSuccess) return e;
+    Probe pr(t, ZHA_K_SEARCH_INIT, st);
+    return launch_chained(search_init_kernel, dim3((unsigned)W), dim3(128), 0, st, ia);
+}
+
+cudaError_t launch_score_level(const zha_tree *t, const Scratch &s, int l, int G, cudaStream_t st) {
+    const zha_config &c = t->cfg;
+    ScoreArgs sa{};
+    sa.nodes = t->nodes[l];
+    sa.node_tree = t->cap_nodes[l] * t->NF;
+    sa.NF = t->NF;
+    sa.R = c.R;
+    sa.G = G;
+    sa.T = t->T;
+    sa.beta = c.sharpness;
+    sa.U = s.U[l];
+    sa.M = s.M[l];
+    sa.words = (t->cap_nodes[l] + 31) / 32;
+    sa.n_level = t->n_nodes[l];
+    sa.qf = s.qf;
+    sa.S = s.S;
+    sa.Sstride = s.Sstride;
+    sa.npi = 4;
+    switch (c.d) {
+        case 64: return launch_score_d<64>(t, sa, st);
+        case 128: return launch_score_d<128>(t, sa, st);
+        default: return launch_score_d<256>(t, sa, st);
     }
+}
+
+cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zha_dtype q_dtype, int G,
+                          long long W, int mode, float p, int k, int *sel, int *sel_count, int max_sel,
+                          zha_stats *stats, int start_level, cudaStream_t st) {
+    const zha_config &c = t->cfg;
+    const int C = c.chunk;
+    cudaError_t e;
+    auto words = [&](int l) { return (t->cap_nodes[l] + 31) / 32; };
+    if ((e = launch_search_init(t, s, Q, q_dtype, G, W, stats, start_level, st)) != cudaSuccess) return e;
 
     // trees walked by many bf16 queries score whole small levels on the tensor cores
     bool tc_any = false;
@@ -888,28 +927,7 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
                                        st);
             if (e != cudaSuccess) return e;
         } else {
-            ScoreArgs sa{};
-            sa.nodes = t->nodes[l];
-            sa.node_tree = t->cap_nodes[l] * t->NF;
-            sa.NF = t->NF;
-            sa.R = c.R;
-            sa.G = G;
-            sa.T = t->T;
-            sa.beta = c.sharpness;
-            sa.U = s.U[l];
-            sa.M = s.M[l];
-            sa.words = words(l);
-            sa.n_level = t->n_nodes[l];
-            sa.qf = s.qf;
-            sa.S = s.S;
-            sa.Sstride = s.Sstride;
-            sa.npi = 4;
-            switch (D) {
-                case 64: e = launch_score_d<64>(t, sa, st); break;
-                case 128: e = launch_score_d<128>(t, sa, st); break;
-                default: e = launch_score_d<256>(t, sa, st); break;
-            }
-            if (e != cudaSuccess) return e;
+            if ((e = launch_score_level(t, s, l, G, st)) != cudaSuccess) return e;
         }
 
         SelectArgs se{};
@@ -964,6 +982,284 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
         cur ^= 1;
     }
     return cudaSuccess;
+}
+
+
+// ---------------------------------------------------------------------------
+// Context-parallel walk: this process holds a shard of every tree (keys
+// key_begin .. of the whole sequence, whole top-level nodes, so its level-l
+// nodes are the whole tree's nodes off_l = key_begin / C^l onward). A level
+// step is: score the shard's frontier (the CUDA-core scorer, as a search
+// does), export each walk's (global id, score) list, let the caller gather the
+// lists of every process (process order = id order), then pack them per walk,
+// choose over them with the selector's list mode (the same passes, so the
+// same choice as one search over the whole tree), and keep the opened nodes
+// the shard holds: their children, and the orphans of the level below (only on
+// the last process), are the shard's next frontier.
+namespace {
+
+struct CpExportArgs {
+    int C, start;
+    long long n_level, n_orph, off;
+    const int *par;
+    long long Lstride;
+    const int *npar;
+    const float *S;
+    long long Sstride;
+    int *ids;
+    float *scores;
+    int *counts;
+    long long stride;
+    int *status;
+};
+
+// one CTA per walk: the shard's frontier in position (= id) order, ids made global
+__global__ void cp_export_kernel(CpExportArgs a) {
+    const long long w = blockIdx.x;
+    const long long npar = a.start ? 0 : a.npar[w];
+    const long long kids = npar * a.C;
+    const long long F = a.start ? a.n_level : kids + a.n_orph;
+    const long long n = F < a.stride ? F : a.stride;
+    if (threadIdx.x == 0) {
+        a.counts[w] = (int)n;
+        if (F > a.stride) report(a.status, DEV_CAPACITY);
+    }
+    const int *par = a.par + w * a.Lstride;
+    for (long long i = threadIdx.x; i < n; i += blockDim.x) {
+        long long id;
+        if (a.start) id = i;
+        else if (i < kids) id = (long long)par[i / a.C] * a.C + i % a.C;
+        else id = (a.n_level - a.n_orph) + (i - kids);
+        a.ids[w * a.stride + i] = (int)(id + a.off);
+        a.scores[w * a.stride + i] = a.S[w * a.Sstride + id];
+    }
+}
+
+// one CTA per walk: the gathered lists of the n_parts processes, concatenated
+__global__ void cp_pack_kernel(int n_parts, const int *ids, const float *scores, const int *counts, long long stride,
+                               long long W, int *pids, float *pscores, int *pcount, long long P) {
+    const long long w = blockIdx.x;
+    long long base = 0;
+    for (int r = 0; r < n_parts; ++r) {
+        long long c = counts[(long long)r * W + w];
+        c = c < 0 ? 0 : (c > stride ? stride : c);
+        const long long src = ((long long)r * W + w) * stride;
+        for (long long i = threadIdx.x; i < c; i += blockDim.x) {
+            pids[w * P + base + i] = ids[src + i];
+            pscores[w * P + base + i] = scores[src + i];
+        }
+        base += c;
+    }
+    if (threadIdx.x == 0) pcount[w] = (int)base;
+}
+
+struct CpLocalArgs {
+    int level, C, G;
+    const int *opened;
+    const int *ocount;
+    long long P;
+    long long lo, n_local;  // the shard's ids at this level: [lo, lo + n_local)
+    // level > 1: the shard's opened nodes (local ids) and the next level's membership bits
+    int *par_out;
+    int *npar_out;
+    long long Lstride;
+    unsigned *M_next, *U_next;
+    long long words_next, n_next_local, n_orph_next;
+    // level 1: the shard's chosen chunks (local ids)
+    int *sel;
+    int *sel_count;
+    int max_sel;
+    int *status;
+};
+
+// one CTA per walk: the opened ids (ascending) that fall in the shard
+__global__ void cp_localize_kernel(CpLocalArgs a) {
+    __shared__ long long s_b0, s_b1;
+    const long long w = blockIdx.x;
+    const int t = (int)(w / a.G), g = (int)(w % a.G);
+    const int *op = a.opened + w * a.P;
+    const long long n = a.ocount[w];
+    if (threadIdx.x == 0) {
+        // first position with id >= lo, first with id >= lo + n_local
+        long long lo = 0, hi = n;
+        while (lo < hi) {
+            const long long mid = (lo + hi) >> 1;
+            if (op[mid] < a.lo) lo = mid + 1;
+            else hi = mid;
+        }
+        s_b0 = lo;
+        hi = n;
+        while (lo < hi) {
+            const long long mid = (lo + hi) >> 1;
+            if (op[mid] < a.lo + a.n_local) lo = mid + 1;
+            else hi = mid;
+        }
+        s_b1 = lo;
+    }
+    __syncthreads();
+    const long long b0 = s_b0, b1 = s_b1;
+    if (a.level > 1) {
+        unsigned *M_tree = a.M_next + (long long)t * a.words_next * a.G;
+        unsigned *U_tree = a.U_next + (long long)t * a.words_next;
+        for (long long i = b0 + threadIdx.x; i < b1; i += blockDim.x) {
+            const long long local = op[i] - a.lo;
+            a.par_out[w * a.Lstride + (i - b0)] = (int)local;
+            set_bits(M_tree, U_tree, a.G, g, local * a.C, local * a.C + a.C);
+        }
+        if (a.n_orph_next > 0) {
+            const long long lo = a.n_next_local - a.n_orph_next, hi = a.n_next_local;
+            for (long long wd = (lo >> 5) + threadIdx.x; wd <= (hi - 1) >> 5; wd += blockDim.x) {
+                const long long wlo = lo > (wd << 5) ? lo : (wd << 5);
+                const long long whi = hi < ((wd + 1) << 5) ? hi : ((wd + 1) << 5);
+                set_bits(M_tree, U_tree, a.G, g, wlo, whi);
+            }
+        }
+        if (threadIdx.x == 0) a.npar_out[w] = (int)(b1 - b0);
+    } else {
+        for (long long i = b0 + threadIdx.x; i < b1 && i - b0 < a.max_sel; i += blockDim.x)
+            a.sel[w * a.max_sel + (i - b0)] = op[i] - (int)a.lo;
+        if (threadIdx.x == 0) {
+            a.sel_count[w] = (int)(b1 - b0 < a.max_sel ? b1 - b0 : a.max_sel);
+            if (b1 - b0 > a.max_sel) report(a.status, DEV_CAPACITY);
+        }
+    }
+}
+
+__global__ void lse_combine_kernel(int n_parts, long long W, int D, const float *outs, const float *lses, void *out,
+                                   int out_bf16, float *lse) {
+    const long long w = blockIdx.x;
+    float m = -INFINITY;
+    for (int r = 0; r < n_parts; ++r) m = fmaxf(m, lses[(long long)r * W + w]);
+    float l = 0.f;
+    for (int r = 0; r < n_parts; ++r) {
+        const float x = lses[(long long)r * W + w];
+        l += x == -INFINITY ? 0.f : expf(x - m);
+    }
+    for (int e = threadIdx.x; e < D; e += blockDim.x) {
+        float acc = 0.f;
+        for (int r = 0; r < n_parts; ++r) {
+            const float x = lses[(long long)r * W + w];
+            if (x != -INFINITY) acc = fmaf(expf(x - m), outs[((long long)r * W + w) * D + e], acc);
+        }
+        const float v = l > 0.f ? acc / l : 0.f;
+        if (out_bf16) static_cast<__nv_bfloat16 *>(out)[w * D + e] = __float2bfloat16_rn(v);
+        else static_cast<float *>(out)[w * D + e] = v;
+    }
+    if (threadIdx.x == 0 && lse) lse[w] = l > 0.f ? m + logf(l) : -INFINITY;
+}
+
+}  // namespace
+
+cudaError_t launch_cp_export(const zha_tree *t, const Scratch &s, int cur, int level, bool start, long long off,
+                             long long W, int *ids, float *scores, int *counts, long long stride, cudaStream_t st) {
+    CpExportArgs a{};
+    a.C = t->cfg.chunk;
+    a.start = start ? 1 : 0;
+    a.n_level = t->n_nodes[level];
+    a.n_orph = start ? 0 : t->n_nodes[level] - (long long)a.C * t->n_nodes[level + 1];
+    a.off = off;
+    a.par = s.L[cur];
+    a.Lstride = s.Lstride;
+    a.npar = s.cnt[cur];
+    a.S = s.S;
+    a.Sstride = s.Sstride;
+    a.ids = ids;
+    a.scores = scores;
+    a.counts = counts;
+    a.stride = stride;
+    a.status = t->d_status;
+    Probe pr(t, ZHA_K_SELECT, st);
+    cp_export_kernel<<<(unsigned)W, 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cp_select(const zha_tree *t, const Scratch &s, int cur, int level, int G, long long W, int n_parts,
+                             const int *ids, const float *scores, const int *counts, long long stride, int mode,
+                             float p, int k, const CpScratch &cs, long long lo, int *sel, int *sel_count,
+                             int max_sel, cudaStream_t st) {
+    const zha_config &c = t->cfg;
+    const long long P = cs.P;
+    cudaError_t e;
+    {
+        Probe pr(t, ZHA_K_SELECT, st);
+        cp_pack_kernel<<<(unsigned)W, 256, 0, st>>>(n_parts, ids, scores, counts, stride, W, cs.pids, cs.pscores,
+                                                     cs.pcount, P);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    SelectArgs se{};
+    se.level = level;
+    se.C = c.chunk;
+    se.c_shift = (c.chunk & (c.chunk - 1)) == 0 ? __builtin_ctz((unsigned)c.chunk) : -1;
+    se.R = c.R;
+    se.G = G;
+    se.start = 0;
+    se.list_ids = cs.pids;
+    se.list_scores = cs.pscores;
+    se.list_count = cs.pcount;
+    se.list_stride = P;
+    se.Sstride = P;  // the global staging rows are P keys long
+    se.gkey = cs.stage;
+    se.mode = mode;
+    se.p = p;
+    se.k = k;
+    if (level > 1) {
+        se.par_out = cs.opened;
+        se.Lstride = P;
+        se.n_par_out = cs.ocount;
+    } else {
+        se.sel = cs.opened;
+        se.max_sel = (int)P;
+        se.sel_count = cs.ocount;
+    }
+    se.status = t->d_status;
+    {
+        Probe pr(t, ZHA_K_SELECT, st);
+        if (P > 8192) {
+            se.smem_keys = std::min<long long>(P, 16384);
+            e = launch_select<1024>(se, W, st);
+        } else if (P > 2048) {
+            se.smem_keys = P;
+            e = launch_select<512>(se, W, st);
+        } else {
+            se.smem_keys = P;
+            e = launch_select<256>(se, W, st);
+        }
+        if (e != cudaSuccess) return e;
+    }
+    CpLocalArgs la{};
+    la.level = level;
+    la.C = c.chunk;
+    la.G = G;
+    la.opened = cs.opened;
+    la.ocount = cs.ocount;
+    la.P = P;
+    la.lo = lo;
+    la.n_local = t->n_nodes[level];
+    if (level > 1) {
+        la.par_out = s.L[cur ^ 1];
+        la.npar_out = s.cnt[cur ^ 1];
+        la.Lstride = s.Lstride;
+        la.M_next = s.M[level - 1];
+        la.U_next = s.U[level - 1];
+        la.words_next = (t->cap_nodes[level - 1] + 31) / 32;
+        la.n_next_local = t->n_nodes[level - 1];
+        la.n_orph_next = t->n_nodes[level - 1] - (long long)c.chunk * t->n_nodes[level];
+    } else {
+        la.sel = sel;
+        la.sel_count = sel_count;
+        la.max_sel = max_sel;
+    }
+    la.status = t->d_status;
+    Probe pr(t, ZHA_K_SELECT, st);
+    cp_localize_kernel<<<(unsigned)W, 256, 0, st>>>(la);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_lse_combine(int n_parts, long long W, int D, const float *outs, const float *lses, void *out,
+                               zha_dtype out_dtype, float *lse, cudaStream_t st) {
+    lse_combine_kernel<<<(unsigned)W, D < 256 ? D : 256, 0, st>>>(n_parts, W, D, outs, lses, out,
+                                                                  out_dtype == ZHA_BF16, lse);
+    return cudaGetLastError();
 }
 
 }  // namespace zha
