@@ -153,3 +153,43 @@ def test_bounded_wait_runs_out_and_is_reported():
     for w in range(len(cnt_a)):
         assert np.array_equal(sel_a[w, : cnt_a[w]], sel_b[w, : cnt_b[w]])
     tree.close()
+
+
+@pytest.mark.parametrize("N", [16427, 70003])
+def test_tensor_core_attention_matches_cuda_cores_and_oracle(N):
+    """Trees of 1,100 bf16 walks take the tensor-core attention (tree-major, per
+    128-key tile against the walks that chose one of its chunks); the same
+    selection with the queries as fp32 takes the CUDA-core attention. Both agree
+    with each other and with the oracle, on trees with a 3-key tail (N not a
+    multiple of 128 or of C), for top-p and top-K selections."""
+    Z = zha()
+    K, V, refs, Q = inputs(N, seed=13)
+    tree = Z.Tree(K, V, refs, N, C, DEPTH, BETA)
+    max_sel = N // C
+    Qh = host64(Q).reshape(-1, D)
+    G = (HQ // H) * NQ
+    otrees = [O.build_tree(host64(K[0, h, :N]), host64(refs[h]), C, DEPTH, BETA, store=O.STORE_F32) for h in range(H)]
+    Kh = [host64(K[0, h, :N]) for h in range(H)]
+    Vh = [host64(V[0, h, :N]) for h in range(H)]
+    for mode, p, k in [(O.TOP_P, 0.9, 0), (O.TOP_K, 0, 8), (O.TOP_P, 0.3, 0)]:
+        sel, cnt, _ = tree.search(Q, mode, p, k, max_sel=max_sel)
+        tree.profile(True)
+        out_tc, lse_tc = tree.attend(Q, sel, cnt, out_dtype=torch.float32)
+        kinds = tree.profile_read()
+        tree.profile(False)
+        assert kinds["attend_combine"][0] > 0 and kinds["attend_partial"][0] > 0, kinds  # the tensor-core path ran
+        out_bf, _ = tree.attend(Q, sel, cnt)  # bf16 output, same path
+        out_cc, lse_cc = tree.attend(Q.float(), sel, cnt, out_dtype=torch.float32)  # CUDA cores
+        tree.sync_status()
+        out_tc, out_cc = host64(out_tc).reshape(-1, D), host64(out_cc).reshape(-1, D)
+        lse_tc, lse_cc = lse_tc.cpu().numpy(), lse_cc.cpu().numpy()
+        err = np.abs(out_tc - out_cc) / np.maximum(1.0, np.abs(out_cc))
+        assert err.max() <= 1e-4, f"tensor-core vs CUDA-core attention: {err.max():.3g}"
+        assert np.abs(lse_tc - lse_cc).max() <= 1e-4 * max(1.0, np.abs(lse_cc).max())
+        assert np.abs(host64(out_bf).reshape(-1, D) - out_tc).max() <= 2 ** -8 * max(1.0, np.abs(out_tc).max())
+        sel_h, cnt_h = sel.cpu().numpy(), cnt.cpu().numpy()
+        for wi in sample_walks():
+            h = wi // G
+            o_out, o_lse = O.attend(Kh[h], Vh[h], Qh[wi], sel_h[wi, : cnt_h[wi]], C, otrees[h].n_nodes[1], BETA)
+            assert_attention_close(out_tc[wi], lse_tc[wi], o_out, o_lse, 3e-3, f"walk {wi}")
+    tree.close()
