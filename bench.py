@@ -679,13 +679,40 @@ def run_prefill(args, dev):
         tensor = {"bound": "tensor", "kernel": "score_tc", "achieved": ach, "peak": bf16_peak, "unit": "TFLOP/s",
                   "frac": ach / bf16_peak if bf16_peak else None, "peak_source": "measured (burst)",
                   "ops_per_step": tc_ops, "ms_per_step": tc_ms}
+    # tensor-core attention (trees of >= 1,024 bf16 walks): per (walk, 128-key tile)
+    # pair the max pass and the accumulate pass each take S = QK^T (2 * 128 * 128
+    # flops per walk row), and P V is taken on the hi and lo parts of P (2 x the same)
+    cpt = 128 // w.chunk
+    pairs = 0
+    for r0 in range(0, Wk, 4096):
+        sl, cn = sel[r0:r0 + 4096], cnt[r0:r0 + 4096]
+        tl = torch.div(sl, cpt, rounding_mode="floor")
+        valid = torch.arange(sl.shape[1], device=sl.device)[None, :] < cn[:, None]
+        first = valid[:, :1] & (cn[:, None] > 0)
+        new = (tl[:, 1:] != tl[:, :-1]) & valid[:, 1:]
+        pairs += int(first.sum().item()) + int(new.sum().item())
+    tail = tree.n_keys - w.chunk * tree.level(1)[1]
+    if tail > 0:
+        pairs += Wk  # every walk reads the tile holding the tail
+    att_ms = kt.get("attend_partial", 0.0)
+    att_flops = pairs * 4 * 2.0 * 128 * 128
+    keys = int(cnt.long().sum().item()) * w.chunk + Wk * tail
+    attention = {"path": "tensor cores (tree-major over 128-key tiles)" if kt.get("attend_combine") else "CUDA cores",
+                 "walk_tile_pairs": pairs, "keys_attended": keys,
+                 "ms": {k2: kt.get(k2) for k2 in ("attend_plan", "attend_partial", "attend_combine")},
+                 "tensor": {"bound": "tensor", "kernel": "atc_max + atc_accum", "achieved":
+                            att_flops / (att_ms / 1e3) / 1e12 if att_ms else None, "peak": bf16_peak,
+                            "unit": "TFLOP/s", "frac": (att_flops / (att_ms / 1e3) / 1e12 / bf16_peak)
+                            if att_ms and bf16_peak else None, "ops_per_step": att_flops,
+                            "what": "MMA work issued: 4 x 2 x 128 x 128 per (walk, tile) pair"},
+                 "algorithmic_tflops": keys * 4.0 * w.d / (att_ms / 1e3) / 1e12 if att_ms else None}
     res = {"workload": f"prefill: {w.queries_per_head:,} queries x 16 q-heads against the 4 KV-head trees of one "
                        "262,144-key sequence, d=128, bf16, C=8, depth 6, R=8, top-p 0.9",
            "walks": Wk, "ms": ms, "value": Wk / (ms / 1e3), "unit": UNIT, "kernel_ms": kt,
            "score_tflops": (flops / ((kt.get("score", 0) + kt.get("score_tc", 0)) / 1e3) / 1e12
                             if kt.get("score") or kt.get("score_tc") else None),
            "scored_walk_nodes": walk_nodes, "union_nodes": sum(info["union_nodes"][1:info["start_level"] + 1]),
-           "tensor_roofline": tensor}
+           "tensor_roofline": tensor, "attention": attention}
     tree.close()
     del inp, sel, cnt, out, lse
     torch.cuda.empty_cache()
