@@ -504,9 +504,24 @@ def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes
             kbytes = B * H * tree.n_keys * d * inp.K.element_size()
             r = results[mname]
             search_ms = sum(r["kernel_ms_per_step"][k2] for k2 in ("search_init", "score", "select", "score_tc"))
+            # the full-scan scorer against its own roofline: every key read once per
+            # tree, every walk's score written once (4 B)
+            peak, peak_kind = peaks()
+            sbytes = kbytes + Wk * tree.n_keys * 4
+            score_ms = dk.get("score")
+            roof_ms = sbytes / (peak * 1e9) * 1e3
             dense[mname] = {"ms": ms, "key_read_gbs": kbytes / (ms / 1e3) / 1e9, "kernel_ms": dk,
                             "keys_selected_mean": float(dcnt.float().mean().item()),
-                            "tree_search_ms": search_ms, "dense_over_tree_search": ms / search_ms}
+                            "tree_search_ms": search_ms, "dense_over_tree_search": ms / search_ms,
+                            "score_roofline": {"bound": "hbm", "kernel": "dense_score", "achieved":
+                                               sbytes / (score_ms / 1e3) / 1e9 if score_ms else None,
+                                               "peak": peak, "unit": "GB/s", "frac": sbytes / (score_ms / 1e3) / 1e9 /
+                                               peak if score_ms else None, "peak_source": peak_kind,
+                                               "bytes_per_launch": sbytes},
+                            "score_at_roofline_ms": roof_ms,
+                            "score_at_roofline_over_tree_search": roof_ms / search_ms,
+                            "what": "score_at_roofline_ms: the full scan's key reads and score writes at the "
+                                    "measured HBM peak, its selection not counted"}
         del dsel, dcnt
         # chunk-mass profile of the same dense attention: per walk, the fewest
         # 16-key chunks holding 90% of it (the statistic the pages quote for real
