@@ -962,19 +962,24 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
         se.status = t->d_status;
         se.gkey = s.gkey;
         {
+            // the widest frontier a walk can have at this level: the whole level, or
+            // for top-K below the start level the children of K nodes and the orphans
+            long long fmax = t->n_nodes[l];
+            if (mode == ZHA_TOP_K && l != start_level)
+                fmax = std::min<long long>(fmax, (long long)k * C + se.n_orph);
             Probe pr(t, ZHA_K_SELECT, st);
-            if (t->n_nodes[l] > 8192) {
+            if (fmax > 8192) {
                 // few walks: the widest frontier sets the time, give it 1,024 threads;
                 // many walks (prefill): 512 threads keep two CTAs per SM
-                se.smem_keys = std::min<long long>(t->n_nodes[l], 16384);
+                se.smem_keys = std::min<long long>(fmax, 16384);
                 e = W <= 2LL * num_sms() ? launch_select<1024>(se, W, st) : launch_select<512>(se, W, st);
-            } else if (t->n_nodes[l] > 2048 && W <= 2LL * num_sms()) {
+            } else if (fmax > 2048 && W <= 2LL * num_sms()) {
                 // few walks over a level of thousands of nodes: frontiers of a few
                 // thousand keys, 512 threads
-                se.smem_keys = t->n_nodes[l];
+                se.smem_keys = fmax;
                 e = launch_select<512>(se, W, st);
             } else {
-                se.smem_keys = t->n_nodes[l];
+                se.smem_keys = fmax;
                 e = launch_select<256>(se, W, st);
             }
             if (e != cudaSuccess) return e;
