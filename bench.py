@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--batch", type=int, default=0, help="sequences per GPU (default: the workload's)")
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the prefill workload and print its line (for profiling)")
+    ap.add_argument("--build-only", action="store_true",
+                    help="build the 256K workload's trees (--batch sequences), time zha_rebuild, print its line")
     ap.add_argument("--parity-trees", type=int, default=4,
                     help="trees per workload whose walks the CPU leg checks against the oracle (0: none)")
     ap.add_argument("--prefill-queries", type=int, default=0,
@@ -765,6 +767,23 @@ def main():
     if args.prefill_only:
         if rank == 0:
             print(json.dumps(run_prefill(args, dev)), flush=True)
+        return
+    if args.build_only:
+        if rank == 0:
+            import tree_indexed_sparse_append_b200 as Z
+
+            w = S.WORKLOADS["kv256k"]
+            if args.batch:
+                w = S.scaled(w, batch=args.batch)
+            w = S.scaled(w, appends=0)
+            inp = S.draw(w, device="cuda")
+            tree = Z.Tree(inp.K, inp.V, inp.refs, w.n_keys, w.chunk, w.depth, w.beta, w.top_width)
+            torch.cuda.synchronize()
+            flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+            line = build_roofline(w, tree, flush, torch.cuda.current_stream(), inp.K.element_size())
+            line["workload"] = f"kv256k build: {w.batch} seq x {w.n_kv_heads} KV heads x {w.n_keys:,} keys"
+            print(json.dumps(line), flush=True)
+            tree.close()
         return
     if world > 1:
         import datetime

@@ -47,10 +47,11 @@ namespace {
 
 constexpr int AT_KEYS = TC_N;  // keys per tile
 constexpr int AT_THREADS = 128;
-// max pass: K tile, queries; accumulate pass: K tile, V^T tile, queries, P hi,
-// P lo; then barriers, the TMEM address and a flag
+// max pass: K tile, queries; accumulate pass: V^T tile, K tile (then P's lo
+// part), queries (then P's hi part), so that two CTAs fit on an SM; then
+// barriers, the TMEM address and a flag
 constexpr int AT_SMEM_MAX = TC_PART + TC_ATILE + 64;
-constexpr int AT_SMEM_ACC = 4 * TC_PART + TC_ATILE + 64;
+constexpr int AT_SMEM_ACC = 2 * TC_PART + TC_ATILE + 64;
 
 struct AtcArgs {
     const __nv_bfloat16 *K, *V, *Q;  // cache [T][cap][128], queries [W][128]
@@ -292,9 +293,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1) atc_max_kernel(AtcArgs a) {
 // values over its chosen keys of the tile, added to its accumulators.
 __global__ void __launch_bounds__(AT_THREADS, 1) atc_accum_kernel(AtcArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
-    unsigned char *sK = smem, *sV = smem + TC_PART, *sA = smem + 2 * TC_PART;
-    unsigned char *sPh = smem + 2 * TC_PART + TC_ATILE, *sPl = sPh + TC_PART;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 4 * TC_PART + TC_ATILE);
+    // the K tile and the queries are read only by the S MMA: once it has completed,
+    // their buffers take P's lo and hi parts; K is gathered again for each batch
+    // (the tile is in L2 by then)
+    unsigned char *sV = smem, *sK = smem + TC_PART, *sA = smem + 2 * TC_PART;
+    unsigned char *sPl = sK, *sPh = sA;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 2 * TC_PART + TC_ATILE);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3);
     volatile int *s_ok = reinterpret_cast<volatile int *>(bars + 4);
     const long long tau = blockIdx.x, t = blockIdx.y;
@@ -317,7 +321,6 @@ __global__ void __launch_bounds__(AT_THREADS, 1) atc_accum_kernel(AtcArgs a) {
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    gather_keys(a, t, tau, sK);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -329,6 +332,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) atc_accum_kernel(AtcArgs a) {
     bool ok = true, v_done = false, s_pending = false, o_pending = false;
     uint32_t phase = 0;
     for (int c0 = 0; c0 < count; c0 += TC_M) {
+        gather_keys(a, t, tau, sK);
         const unsigned e = gather_queries(a, t, list, c0, count, sA);
         cp_async_wait_all();
         __syncthreads();
