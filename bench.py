@@ -600,7 +600,9 @@ def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes
             walks = sum(len(v[3]) for v in sample.values())
             used = min(cores, walks)
             v, done = oracle_walks_per_second(w, sample, args.cpu_seconds, used)
+            v1, done1 = oracle_walks_per_second(w, sample, max(1.0, args.cpu_seconds / 4), 1)
             baseline = {"value": v, "unit": UNIT, "cores": used, "cpu_model": cpu_model(), "kind": "oracle",
+                        "single_thread": {"value": v1, "walks": done1},
                         "sample": f"{n_trees} of {w.trees} trees ({walks} walks), append + search + attend per "
                                   f"step, {done} walks in {args.cpu_seconds:.0f} s, oracle trees built beforehand",
                         "oracle_build_s": build_s,

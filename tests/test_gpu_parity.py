@@ -492,7 +492,7 @@ def test_chunk_mass_matches_oracle(N, d, dtype, Hq, nq, group):
 @pytest.mark.parametrize("dtype,d,C,depth", [(torch.float32, 64, 4, 4), (torch.bfloat16, 128, 8, 3)])
 def test_ref_grad_matches_oracle(dtype, d, C, depth):
     """The split loss and its gradient with respect to the references against the
-    CPU reference (explicit backward in double precision)."""
+    CPU reference (explicit backward in double precision), to what fp32 gives."""
     from oracle import ref_learning as RL
 
     Z = zha()
@@ -512,10 +512,13 @@ def test_ref_grad_matches_oracle(dtype, d, C, depth):
         lo, go = RL.split_loss_and_grad(host64(K[0, h, :N]), host64(refs[h]), q, C, depth, beta)
         losses.append(lo)
         grads.append(go / H)  # the GPU averages over all walks of all trees
-    assert abs(loss - np.mean(losses)) <= 2e-4 * max(1.0, abs(np.mean(losses))), (loss, losses)
-    for h in range(H):
-        scale = max(1e-6, np.abs(grads[h]).max())
-        assert np.abs(grad[h] - grads[h]).max() <= 2e-3 * scale, (h, np.abs(grad[h] - grads[h]).max(), scale)
+    loss_err = abs(loss - np.mean(losses)) / max(1.0, abs(np.mean(losses)))
+    grad_err = max(np.abs(grad[h] - grads[h]).max() / max(1e-6, np.abs(grads[h]).max()) for h in range(H))
+    print(f"ref_grad {dtype}: loss error {loss_err:.3g}, gradient error {grad_err:.3g} of its largest element")
+    # fp32 arithmetic over sums of a few thousand terms: observed on B200 1.4e-7 on
+    # the loss and 9e-7 (fp32 caches) / 1.5e-6 (bf16) of the largest gradient element
+    assert loss_err <= 2e-6, (loss, losses)
+    assert grad_err <= 2e-5, grad_err
     tree.close()
 
 
