@@ -11,8 +11,14 @@
 //
 // Mapping (all arithmetic fp32; the softmax is taken online over batches of
 // children, so a node's children are read once):
-//   build_leaf_kernel   level 1: a warp per node (a contiguous run of nodes per
-//                       warp), its references RPW at a time (4 at D = 128). Lane
+//   build_leaf_batch_kernel  level 1 (C a power of two up to 32, R <= 8): a warp
+//                       per batch of 32 keys, lane i scoring key i whole against
+//                       references broadcast from shared memory, then lanes
+//                       summing column slices of the weighted keys (described
+//                       at the kernel).
+//   build_leaf_kernel   level 1 otherwise: a warp per node (a contiguous run of
+//                       nodes per warp), its references RPW at a time (4 at
+//                       D = 128). Lane
 //                       l owns D/32 consecutive columns of each key; the node's
 //                       keys are loaded together (all loads in flight at once)
 //                       and kept for every reference group, each key's RPW dot
@@ -310,6 +316,198 @@ __global__ void __launch_bounds__(256, 2) build_leaf_kernel(BuildArgs a) {
     chain_done();
 }
 
+// Eight consecutive key elements from shared memory as floats (one 16-byte load
+// for bf16, two for fp32).
+template <typename KT>
+__device__ __forceinline__ void lds8(const char *p, float (&v)[8]);
+template <>
+__device__ __forceinline__ void lds8<__nv_bfloat16>(const char *p, float (&v)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const unsigned w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+template <>
+__device__ __forceinline__ void lds8<float>(const char *p, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4 *>(p);
+    const float4 b = *reinterpret_cast<const float4 *>(p + 16);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+constexpr int LEAF_RP = 8;  // references per pass of the batch kernel (R <= 8)
+
+// Shared memory of one warp of build_leaf_batch_kernel: the batch's 32 key rows
+// (padded by 16 bytes), the references transposed ([D][8] fp32) and the weights
+// ([32 keys][8] fp32).
+template <typename KT, int D>
+struct LeafSmem {
+    static constexpr int ROW = D * (int)sizeof(KT) + 16;
+    static constexpr int KEYS = 32 * ROW;
+    static constexpr int REFS = D * LEAF_RP * 4;
+    static constexpr int WTS = 32 * LEAF_RP * 4;
+    static constexpr int BYTES = KEYS + REFS + WTS;
+};
+
+// Level-1 nodes, one warp per batch of 32 consecutive keys: 32 / C nodes of one
+// tree (C a power of two, 2..32; R <= 8). Each warp takes a contiguous run of the
+// batches (tree-major).
+//   1. The batch's keys are copied to the warp's shared memory with coalesced
+//      16-byte loads (rows padded by 16 bytes, so lanes reading different rows
+//      use different banks).
+//   2. Lane i takes key i whole: its 8 dot products with the references (kept
+//      transposed in shared memory and read by broadcast) need no reduction across
+//      lanes. The softmax and log-sum-exp over a node's children are taken across
+//      the C lanes of its keys (xor shuffles inside the group).
+//   3. Lane l then takes 8 columns of one node (D / 8 lanes per node) and sums the
+//      node's weighted keys for all 8 references from the staged rows.
+// With key_r = sum_i w_i k_i, beta <key_r, q_r> = sum_i w_i s_i, so
+// bias_r = lse_r - sum_i w_i s_i = sum_i w_i (log z_r - (s_i - m_r)) (m_r the
+// largest score, z_r the sum of exp(s_i - m_r)): no second dot product, and no
+// difference of two large terms.
+template <typename KT, int D>
+__global__ void __launch_bounds__(256) build_leaf_batch_kernel(BuildArgs a) {
+    chain_start();
+    using SM = LeafSmem<KT, D>;
+    constexpr int PPR = D * (int)sizeof(KT) / 16;  // 16-byte pieces per key row
+    constexpr int LPN = D / 8;                      // lanes per node in step 3
+    constexpr int NPP = 32 / LPN > 0 ? 32 / LPN : 1;
+    static_assert(LPN <= 32, "D <= 256");
+    extern __shared__ __align__(16) char leaf_smem[];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    char *s_keys = leaf_smem + (size_t)wid * SM::BYTES;
+    float *s_ref = reinterpret_cast<float *>(s_keys + SM::KEYS);
+    float *s_w = s_ref + D * LEAF_RP;
+
+    const int C = a.C, NPW = 32 / a.C;
+    const long long bpt = (a.per_tree + NPW - 1) / NPW;  // batches per tree
+    const long long batches = (a.items / a.per_tree) * bpt;
+    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+    const long long per_warp = (batches + nw - 1) / nw;
+    long long b = gw * per_warp;
+    const long long b_end = b + per_warp < batches ? b + per_warp : batches;
+    const KT *K = static_cast<const KT *>(a.child);
+    int cur_h = -1;
+    for (; b < b_end; ++b) {
+        const long long t = b / bpt, bj = b - t * bpt;
+        const int h = (int)(t % a.H_kv);
+        const long long j = a.j0 + bj * NPW;  // first node of the batch
+        const long long left = a.per_tree - bj * NPW;
+        const int nb = left < NPW ? (int)left : NPW;  // nodes in the batch
+        const int nk = nb * C;
+
+        __syncwarp();  // the previous batch's rows and weights are no longer read
+        if (h != cur_h) {
+            const float *q = a.refs + (long long)h * a.R * D;
+            for (int idx = lane; idx < LEAF_RP * D; idx += 32) {
+                const int r = idx / D, c = idx - r * D;
+                s_ref[c * LEAF_RP + r] = r < a.R ? __ldg(q + idx) : 0.f;
+            }
+            cur_h = h;
+        }
+        // 1. the batch's keys, coalesced
+        {
+            const char *src = reinterpret_cast<const char *>(K + t * a.child_tree + j * C * (long long)D);
+#pragma unroll 4
+            for (int p = lane; p < 32 * PPR; p += 32) {
+                const int key = p / PPR, col = p - key * PPR;
+                if (key < nk) {
+                    const uint4 v = ld_stream_u4(src + (size_t)p * 16);
+                    *reinterpret_cast<uint4 *>(s_keys + key * SM::ROW + col * 16) = v;
+                }
+            }
+        }
+        __syncwarp();
+
+        // 2. lane i: key i's scores against the 8 references
+        float s[LEAF_RP];
+#pragma unroll
+        for (int r = 0; r < LEAF_RP; ++r) s[r] = 0.f;
+        {
+            const char *row = s_keys + lane * SM::ROW;
+#pragma unroll 2
+            for (int c = 0; c < D; c += 8) {
+                float kf[8];
+                lds8<KT>(row + c * (int)sizeof(KT), kf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float4 q0 = *reinterpret_cast<const float4 *>(s_ref + (c + e) * LEAF_RP);
+                    const float4 q1 = *reinterpret_cast<const float4 *>(s_ref + (c + e) * LEAF_RP + 4);
+                    s[0] = fmaf(kf[e], q0.x, s[0]);
+                    s[1] = fmaf(kf[e], q0.y, s[1]);
+                    s[2] = fmaf(kf[e], q0.z, s[2]);
+                    s[3] = fmaf(kf[e], q0.w, s[3]);
+                    s[4] = fmaf(kf[e], q1.x, s[4]);
+                    s[5] = fmaf(kf[e], q1.y, s[5]);
+                    s[6] = fmaf(kf[e], q1.z, s[6]);
+                    s[7] = fmaf(kf[e], q1.w, s[7]);
+                }
+            }
+        }
+        // softmax and log-sum-exp over the node's C lanes (lanes of keys past the
+        // batch compute values that are never stored)
+        float w[LEAF_RP], bias[LEAF_RP];
+#pragma unroll
+        for (int r = 0; r < LEAF_RP; ++r) {
+            const float sr = a.beta * s[r];
+            float m = sr;
+            for (int o = C >> 1; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+            const float e = expf(sr - m);
+            float z = e;
+            for (int o = C >> 1; o >= 1; o >>= 1) z += __shfl_xor_sync(FULL, z, o);
+            w[r] = e / z;
+            float ent = w[r] * (logf(z) - (sr - m));
+            for (int o = C >> 1; o >= 1; o >>= 1) ent += __shfl_xor_sync(FULL, ent, o);
+            bias[r] = ent;
+        }
+        *reinterpret_cast<float4 *>(s_w + lane * LEAF_RP) = make_float4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<float4 *>(s_w + lane * LEAF_RP + 4) = make_float4(w[4], w[5], w[6], w[7]);
+        if ((lane & (C - 1)) == 0 && lane < nk) {
+            float *node = a.out + t * a.out_tree + (j + lane / C) * a.NF;
+#pragma unroll
+            for (int r = 0; r < LEAF_RP; ++r)
+                if (r < a.R) node[(long long)a.R * D + r] = bias[r];
+        }
+        __syncwarp();
+
+        // 3. lane l: columns cs .. cs + 7 of node n, all references
+        const int cs = (lane % LPN) * 8;
+        for (int n = lane / LPN; n < nb; n += NPP) {
+            float o[LEAF_RP][8];
+#pragma unroll
+            for (int r = 0; r < LEAF_RP; ++r)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[r][e] = 0.f;
+#pragma unroll 2
+            for (int i = 0; i < C; ++i) {
+                const int key = n * C + i;
+                float kf[8];
+                lds8<KT>(s_keys + key * SM::ROW + cs * (int)sizeof(KT), kf);
+                const float4 w0 = *reinterpret_cast<const float4 *>(s_w + key * LEAF_RP);
+                const float4 w1 = *reinterpret_cast<const float4 *>(s_w + key * LEAF_RP + 4);
+                const float wr[LEAF_RP] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                for (int r = 0; r < LEAF_RP; ++r)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o[r][e] = fmaf(wr[r], kf[e], o[r][e]);
+            }
+            float *node = a.out + t * a.out_tree + (j + n) * a.NF + cs;
+#pragma unroll
+            for (int r = 0; r < LEAF_RP; ++r) {
+                if (r < a.R) {
+                    *reinterpret_cast<float4 *>(node + r * D) = make_float4(o[r][0], o[r][1], o[r][2], o[r][3]);
+                    *reinterpret_cast<float4 *>(node + r * D + 4) = make_float4(o[r][4], o[r][5], o[r][6], o[r][7]);
+                }
+            }
+        }
+    }
+    chain_done();
+}
+
 // Levels >= 2, one warp per (node, reference r): row r of each child, CB at a
 // time (CB * D / 32 registers of rows per lane).
 template <int D>
@@ -428,8 +626,38 @@ inline long long warp_blocks(long long warp_items) {
     return blocks < 1 ? 1 : (blocks > cap ? cap : blocks);
 }
 
+// Warps per block of the batch kernel, and its resident blocks per SM (computed once).
+template <typename KT, int D>
+struct LeafLaunch {
+    int warps = 0, per_sm = 0;
+    cudaError_t err = cudaSuccess;
+    LeafLaunch() {
+        constexpr int per_warp = LeafSmem<KT, D>::BYTES;
+        warps = 8 * per_warp <= 112 * 1024 ? 8 : 4;
+        const int smem = warps * per_warp;
+        err = cudaFuncSetAttribute(build_leaf_batch_kernel<KT, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (err == cudaSuccess)
+            err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, build_leaf_batch_kernel<KT, D>, 32 * warps,
+                                                                smem);
+        if (per_sm < 1) per_sm = 1;
+    }
+};
+
 template <typename KT, int D>
 cudaError_t launch_leaf(const zha_tree *t, const BuildArgs &a, cudaStream_t st) {
+    if (a.R <= LEAF_RP && a.C >= 2 && a.C <= 32 && (a.C & (a.C - 1)) == 0) {
+        static const LeafLaunch<KT, D> L;
+        if (L.err != cudaSuccess) return L.err;
+        const int npw = 32 / a.C;
+        const long long batches = (a.items / a.per_tree) * ((a.per_tree + npw - 1) / npw);
+        long long blocks = (batches + L.warps - 1) / L.warps;
+        const long long cap = (long long)num_sms() * L.per_sm;
+        if (blocks > cap) blocks = cap;
+        if (blocks < 1) blocks = 1;
+        Probe pr(t, ZHA_K_BUILD, st);
+        return launch_chained(build_leaf_batch_kernel<KT, D>, dim3((unsigned)blocks), dim3(32 * L.warps),
+                              (size_t)L.warps * LeafSmem<KT, D>::BYTES, st, a);
+    }
     // RPW references at a time: RPW * D / 32 = 16 registers of references (fewer when R is small)
     constexpr int RPW = 16 / (D / 32);
     const dim3 grid((unsigned)warp_blocks(a.items));
