@@ -429,7 +429,7 @@ def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes
         # profiled pass: per-kernel device time and the frontier sizes behind it
         tree.profile(True)
         kt = {}
-        score_bytes = attend_bytes = walk_keys = 0
+        score_bytes = attend_bytes = walk_keys = walk_nodes = 0
         levels = w.depth
         NF = w.R * w.d + ((w.R + 3) & ~3)
         for i in range(args.profile_steps):
@@ -451,8 +451,18 @@ def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes
             elt = 2 if w.kv_dtype == "bf16" else 4
             attend_bytes += keys * 2 * d * elt + Wk * d * (elt + 4)
             walk_keys += int(c.sum()) * w.chunk + Wk * tail
+            walk_nodes += sum(info["walk_nodes"][1:levels + 1])
         for name, (n, ms) in tree.profile_read().items():
             kt[name] = {"launches": n, "ms": ms}
+        tree.profile(False)
+        # the selector against its fixed cost: the same searches at top-K 1, where
+        # every frontier below the start level holds C nodes (search only)
+        tree.profile(True)
+        n_floor = 5
+        for _ in range(n_floor):
+            flush.zero_()
+            tree.search(inp.Q, Z.TOP_K, 0.0, 1, max_sel=max_sel, out=(sel, cnt, None))
+        floor_ms = tree.profile_read()["select"][1] / n_floor
         tree.profile(False)
         peak, peak_kind = peaks()
         sc = kt["score"]
@@ -470,10 +480,20 @@ def run_decode(w, args, rank, world, dev, with_baseline: bool, label: str, modes
                        "launch_ms": ap["ms"] / max(1, ap["launches"]), "traffic": committed_traffic("attend", label)}
         step_ms = sum(v["ms"] for v in kt.values()) / max(1, args.profile_steps)
         keys_per_walk = walk_keys / max(1, args.profile_steps * Wk)
+        sel_ms = kt["select"]["ms"] / max(1, args.profile_steps)
+        nodes_step = walk_nodes / max(1, args.profile_steps)
+        select = {"bound": "latency", "ms_per_step": sel_ms, "levels": levels,
+                  "floor_ms_per_step": floor_ms, "frontier_ms_per_step": sel_ms - floor_ms,
+                  "walk_nodes_per_step": nodes_step, "score_bytes_per_step": 4 * nodes_step,
+                  "what": "floor: the same trees and queries at top-K 1 (frontiers below the start level C "
+                          "nodes wide), the selector's fixed cost over the levels; frontier_ms: the rest, "
+                          "which grows with the widest frontier of each level; score bytes: 4 B per "
+                          "frontier node of every walk, read from L2-resident score rows"}
         results[mname] = {"qps": qps, "ms_per_step": total_ms / steps, "launches": launches / steps,
                           "keys_per_walk": keys_per_walk, "selected_keys_per_s": qps * keys_per_walk,
                           "context_keys_per_s": qps * tree.n_keys,
                           "clocks": clk.summary(), "roofline": roof, "attend_roofline": attend_roof,
+                          "select": select,
                           "kernel_ms_per_step": {kk: v["ms"] / max(1, args.profile_steps) for kk, v in kt.items()},
                           "kernel_sum_ms_per_step": step_ms, "levels_walked": levels}
 
@@ -807,7 +827,7 @@ def main():
                  "modes": {m: {"value": r["qps"], "ms_per_step": r["ms_per_step"], "roofline": r["roofline"],
                                "keys_per_walk": r["keys_per_walk"], "selected_keys_per_s": r["selected_keys_per_s"],
                                "context_keys_per_s": r["context_keys_per_s"],
-                               "attend_roofline": r["attend_roofline"],
+                               "attend_roofline": r["attend_roofline"], "select": r["select"],
                                "kernel_ms_per_step": r["kernel_ms_per_step"], "clocks": r["clocks"]}
                            for m, r in x["results"].items()},
                  "e2e": x["e2e"], "dense_scan": x["dense"]}
@@ -820,7 +840,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": config_of(head["w"], label),
-        "roofline": r["roofline"], "attend_roofline": r["attend_roofline"],
+        "roofline": r["roofline"], "attend_roofline": r["attend_roofline"], "select": r["select"],
         "cpu_baseline": head["baseline"], "e2e": head["e2e"], "gpu_launches": round(r["launches"] * args.steps),
         "clocks": r["clocks"], "kernel_ms_per_step": r["kernel_ms_per_step"],
         "keys_per_walk": r["keys_per_walk"], "selected_keys_per_s": r["selected_keys_per_s"],

@@ -21,8 +21,9 @@
 //                Each node (R*d fp32 keys + R biases, 4 KB at R=8, d=128) is
 //                streamed from HBM once with 128-bit L1-bypassing loads and
 //                scored against every walk whose frontier holds it (a ballot over
-//                per-walk membership bits). Dot products reduce with a warp
-//                transpose-reduce (R rows in R-1+5-log2 R shuffles).
+//                per-walk membership bits; for trees of at most 4 walks their
+//                queries are loaded with the node). Dot products reduce with a
+//                warp transpose-reduce (R rows in R-1+5-log2 R shuffles).
 //   select_level One CTA per walk. Exact selection without sorting: histogram
 //                passes over 256 buckets (1/8-nat buckets below the frontier's
 //                maximum, then 1/2048-nat buckets inside the crossing one, then
@@ -278,6 +279,35 @@ __device__ __forceinline__ void score_node(const ScoreArgs &a, int t, long long 
     }
 }
 
+// Scores one node (rows in kr) against the walks of tree t whose frontier holds
+// node j, for trees of at most GQ walks whose queries (q[g], this lane's columns)
+// were loaded together with the node: no query load waits on the membership.
+template <int D, int RP, int GQ>
+__device__ __forceinline__ void score_node_q(const ScoreArgs &a, int t, long long j, const float (&kr)[RP][D / 32],
+                                             const float (&q)[GQ][D / 32], float bias, int lane, unsigned mw) {
+    constexpr int EPL = D / 32;
+    constexpr int LG = ilog2(RP);
+    const int rr = lane >> (5 - LG);
+    const unsigned members = __ballot_sync(FULL, (mw >> (j & 31)) & 1u);
+#pragma unroll
+    for (int g = 0; g < GQ; ++g) {
+        if (!((members >> g) & 1u)) continue;
+        float part[RP];
+#pragma unroll
+        for (int r = 0; r < RP; ++r) {
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) s = fmaf(kr[r][e], q[g][e], s);
+            part[r] = s;
+        }
+        const float dot = transpose_reduce<RP>(part, lane);
+        float sc = rr < a.R ? fmaf(a.beta, dot, bias) : -INFINITY;
+#pragma unroll
+        for (int off = 16; off >= (32 >> LG) && LG > 0; off >>= 1) sc = fmaxf(sc, __shfl_xor_sync(FULL, sc, off));
+        if (lane == 0) a.S[((long long)t * a.G + g) * a.Sstride + j] = sc;
+    }
+}
+
 // Grid-stride over (tree, group of npi node ids) items of the level's union
 // bitmap (npi = 4, or 1 for levels too small to give every warp several items).
 // Each lane fetches the union bits of one of the warp's next 32 items in a single
@@ -320,7 +350,25 @@ __global__ void __launch_bounds__(256, 3) score_level_kernel(ScoreArgs a) {
                 float kr[RP][D / 32];
                 load_node<D, RP>(node, a.R, lane, kr);
                 const float bias = rr < a.R ? __ldg(node + a.R * D + rr) : 0.f;
-                score_node<D, RP>(a, t, j, kr, bias, lane);
+                if (a.G <= 4) {
+                    // the tree's queries and membership words, issued with the node
+                    constexpr int EPL = D / 32;
+                    float q[4][EPL];
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        if (g < a.G) {
+                            load_q<EPL>(a.qf + ((long long)t * a.G + g) * D + lane * EPL, q[g]);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < EPL; ++e) q[g][e] = 0.f;
+                        }
+                    }
+                    const unsigned mw =
+                        lane < a.G ? __ldg(a.M + ((long long)t * a.words + (j >> 5)) * a.G + lane) : 0u;
+                    score_node_q<D, RP, 4>(a, t, j, kr, q, bias, lane, mw);
+                } else {
+                    score_node<D, RP>(a, t, j, kr, bias, lane);
+                }
             }
         }
     }
