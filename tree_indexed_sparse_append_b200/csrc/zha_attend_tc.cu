@@ -95,7 +95,10 @@ __global__ void atc_scatter_kernel(AtcArgs a, const int *sel, const int *sel_cou
             report(a.status, DEV_BAD_INDEX);
             continue;
         }
-        atomicOr(&a.bits[(t * a.words1 + (c >> 5)) * a.G + g], 1u << (c & 31));
+        // a reduction without a returned value: nothing waits for it
+        asm volatile("red.relaxed.gpu.global.or.b32 [%0], %1;" ::"l"(&a.bits[(t * a.words1 + (c >> 5)) * a.G + g]),
+                     "r"(1u << (c & 31))
+                     : "memory");
     }
 }
 

@@ -35,6 +35,10 @@
 //                compacted in id order by block scans; their children and the
 //                orphans of the level below form the next frontier (membership
 //                bits per walk and a per-tree union).
+//   select_warp_kernel  Levels whose frontiers hold at most 64 nodes (start
+//                levels of 64 nodes or fewer): one warp per walk, keys in
+//                registers, a bitonic sort across the warp, the same cutoff rule
+//                and the same fixed-point masses, so it opens the same nodes.
 #include <algorithm>
 #include <cmath>
 
@@ -140,6 +144,12 @@ __device__ __forceinline__ void load_q(const float *p, float (&v)[EPL]) {
     }
 }
 
+// OR without a returned value: a reduction the issuing thread does not wait for
+// (many walks set bits in the same union words, so these are contended).
+__device__ __forceinline__ void red_or(unsigned *p, unsigned v) {
+    asm volatile("red.relaxed.gpu.global.or.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Sets bits [lo, hi) of one walk's membership row and of its tree's union.
 __device__ __forceinline__ void set_bits(unsigned *M_tree, unsigned *U_tree, int G, int g, long long lo,
                                          long long hi) {
@@ -148,8 +158,8 @@ __device__ __forceinline__ void set_bits(unsigned *M_tree, unsigned *U_tree, int
         const long long b1 = hi < ((w + 1) << 5) ? hi : ((w + 1) << 5);
         const int n = (int)(b1 - b0);
         const unsigned mask = (n == 32 ? FULL : ((1u << n) - 1u)) << (int)(b0 - (w << 5));
-        atomicOr(&M_tree[w * G + g], mask);
-        atomicOr(&U_tree[w], mask);
+        red_or(&M_tree[w * G + g], mask);
+        red_or(&U_tree[w], mask);
     }
 }
 
@@ -411,6 +421,7 @@ struct SelectArgs {
     const float *list_scores;
     const int *list_count;
     long long list_stride;
+    long long n_walks;       // walks of the call (select_warp_kernel)
 };
 
 // frontier position -> node id (positions and ids fit in 32 bits); lid: the
@@ -803,6 +814,253 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
     chain_done();
 }
 
+// Sorts the 32 * E keys of a warp in descending order (lane l holds positions
+// l * E .. l * E + E - 1): a bitonic network, exchanges across lanes by shuffle
+// and inside a lane in registers.
+template <int E>
+__device__ __forceinline__ void warp_sort_desc(uint32_t (&v)[E], int lane) {
+    constexpr int N = 32 * E;
+#pragma unroll
+    for (int k = 2; k <= N; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j >= 1; j >>= 1) {
+            if (j >= E) {
+                const int lj = j / E;  // partner lane distance
+                const bool lower = (lane & lj) == 0;
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const bool desc = ((lane * E + e) & k) == 0;  // this run sorts descending
+                    const uint32_t o = __shfl_xor_sync(FULL, v[e], lj);
+                    v[e] = lower == desc ? max(v[e], o) : min(v[e], o);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    if ((e & j) == 0) {
+                        const bool desc = ((lane * E + e) & k) == 0;
+                        const uint32_t x = v[e], y = v[e | j];
+                        v[e] = desc ? max(x, y) : min(x, y);
+                        v[e | j] = desc ? min(x, y) : max(x, y);
+                    }
+                }
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long x) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(FULL, x, o);
+    return x;
+}
+
+// One warp per walk, for levels whose frontiers hold at most 32 * E nodes (the
+// host bounds them): the frontier's keys sit in registers (E per lane, in
+// position order), a sorted copy gives the cutoff key kstar as the first key at
+// which the prefix of the fixed-point masses (counts for top-K) reaches the
+// target, and the opened nodes follow the rule of select_level_kernel: keys above
+// kstar, then the first cstar keys equal to it by position. Masses, target and
+// rule are those of the block path, so both choose the same nodes; this one needs
+// no block barrier, and many walks share an SM.
+template <int E>
+__global__ void __launch_bounds__(256) select_warp_kernel(SelectArgs a) {
+    chain_start();
+    const int lane = threadIdx.x & 31;
+    const long long walk = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (walk < a.n_walks) {
+        const int t = (int)(walk / a.G), g = (int)(walk % a.G);
+        const long long npar = a.start ? 0 : a.n_par_in[walk];
+        const int *par = a.start ? nullptr : a.par_in + walk * a.Lstride;
+        long long F = a.start ? a.n_level : npar * a.C + a.n_orph;
+        if (F > 32 * E) {  // outside the host's bound: report, open nothing
+            if (lane == 0) report(a.status, DEV_BAD_INDEX);
+            F = 0;
+        }
+        const float *S = a.S + walk * a.Sstride;
+        // keys in position order (0 past the frontier: below every score's key).
+        // Every load is issued unconditionally at a clamped index, so all E of a
+        // lane are in flight together; positions past the frontier are masked.
+        uint32_t key[E];
+        int id[E];
+        if (a.start) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) id[e] = lane * E + e;
+        } else {
+            const int kids = (int)npar * a.C, C = a.C;
+            const int orph0 = (int)(a.n_level - a.n_orph) - kids;  // id of position i >= kids: orph0 + i
+            int pv[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int i = lane * E + e;
+                const int pi = i < kids ? (a.c_shift >= 0 ? i >> a.c_shift : i / C) : 0;
+                pv[e] = par[pi];  // par holds at least one entry per walk
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int i = lane * E + e;
+                const int pi = a.c_shift >= 0 ? i >> a.c_shift : i / C;
+                id[e] = i < kids ? pv[e] * C + (i - pi * C) : orph0 + i;
+            }
+        }
+        float sv[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) sv[e] = S[lane * E + e < F ? id[e] : 0];
+#pragma unroll
+        for (int e = 0; e < E; ++e) key[e] = lane * E + e < F ? order_key(sv[e]) : 0u;
+        uint32_t kmax = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) kmax = max(kmax, key[e]);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) kmax = max(kmax, __shfl_xor_sync(FULL, kmax, o));
+        const float m = key_to_float(kmax);
+        const bool top_p = a.mode == ZHA_TOP_P;
+        const bool open_all = (top_p && a.p >= 1.f) || (!top_p && (long long)a.k >= F);
+        auto weight = [&](uint32_t k) -> unsigned long long {
+            return k == 0u ? 0ull : (top_p ? mass_fixed(expf(key_to_float(k) - m)) : 1ull);
+        };
+
+        uint32_t kstar = 0;
+        unsigned long long cstar = 0;
+        if (F > 0 && !open_all) {
+            uint32_t sk[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) sk[e] = key[e];
+            warp_sort_desc<E>(sk, lane);
+            unsigned long long w[E], lane_tot = 0;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                w[e] = weight(sk[e]);
+                lane_tot += w[e];
+            }
+            // exclusive prefix of the lanes' totals
+            unsigned long long incl = lane_tot;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long y = __shfl_up_sync(FULL, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const unsigned long long total = __shfl_sync(FULL, incl, 31);
+            unsigned long long target;
+            if (top_p) {
+                target = (unsigned long long)ceil((double)a.p * (double)total);
+                if (target < 1) target = 1;
+                if (target > total) target = total;
+            } else {
+                target = (unsigned long long)a.k;
+            }
+            // the cutoff: the sorted key whose weight takes the prefix to the target
+            unsigned long long pre = incl - lane_tot;
+            uint32_t mine = 0;
+            bool hit = false;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                if (!hit && pre < target && target <= pre + w[e]) {
+                    hit = true;
+                    mine = sk[e];
+                }
+                pre += w[e];
+            }
+            const unsigned hb = __ballot_sync(FULL, hit);
+            kstar = __shfl_sync(FULL, mine, hb ? __ffs(hb) - 1 : 0);
+            // weight strictly above kstar, then how many of its equal keys to open
+            unsigned long long above = 0;
+#pragma unroll
+            for (int e = 0; e < E; ++e) above += sk[e] > kstar ? w[e] : 0ull;
+            above = warp_sum_u64(above);
+            const unsigned long long u = weight(kstar);
+            const unsigned long long rem = target > above ? target - above : 0ull;
+            cstar = top_p ? (u > 0 ? (rem + u - 1) / u : 1ull) : rem;
+        }
+
+        // opened positions, in position order: rank among the keys equal to kstar
+        // by a scan of per-lane counts, then compaction by a scan of opened counts
+        bool open[E];
+        {
+            unsigned eq_l = 0;
+#pragma unroll
+            for (int e = 0; e < E; ++e) eq_l += (key[e] == kstar && key[e] != 0u) ? 1u : 0u;
+            unsigned eq_incl = eq_l;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned y = __shfl_up_sync(FULL, eq_incl, o);
+                if (lane >= o) eq_incl += y;
+            }
+            unsigned eq = eq_incl - eq_l;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const bool in = lane * E + e < F;
+                if (open_all) {
+                    open[e] = in;
+                } else {
+                    const bool is_eq = in && key[e] == kstar;
+                    open[e] = in && (key[e] > kstar || (is_eq && (unsigned long long)eq < cstar));
+                    eq += is_eq ? 1u : 0u;
+                }
+            }
+        }
+        unsigned n_l = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) n_l += open[e] ? 1u : 0u;
+        unsigned n_incl = n_l;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned y = __shfl_up_sync(FULL, n_incl, o);
+            if (lane >= o) n_incl += y;
+        }
+        const unsigned n_open = __shfl_sync(FULL, n_incl, 31);
+        unsigned r = n_incl - n_l;
+        unsigned *M_tree = a.M_next ? a.M_next + (long long)t * a.words_next * a.G : nullptr;
+        unsigned *U_tree = a.U_next ? a.U_next + (long long)t * a.words_next : nullptr;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            if (!open[e]) continue;
+            const long long nid = id[e];
+            if (a.level == 1) {
+                if (r < (unsigned)a.max_sel) a.sel[walk * a.max_sel + r] = (int)nid;
+            } else {
+                a.par_out[walk * a.Lstride + r] = (int)nid;
+                if (M_tree) set_bits(M_tree, U_tree, a.G, g, nid * a.C, nid * a.C + a.C);
+            }
+            ++r;
+        }
+        if (a.level > 1 && a.n_orph_next > 0 && M_tree) {
+            const long long lo = a.n_level_next - a.n_orph_next, hi = a.n_level_next;
+            for (long long wd = (lo >> 5) + lane; wd <= (hi - 1) >> 5; wd += 32) {
+                const long long wlo = lo > (wd << 5) ? lo : (wd << 5);
+                const long long whi = hi < ((wd + 1) << 5) ? hi : ((wd + 1) << 5);
+                set_bits(M_tree, U_tree, a.G, g, wlo, whi);
+            }
+        }
+        if (lane == 0) {
+            if (a.level > 1) {
+                a.n_par_out[walk] = (int)n_open;
+            } else {
+                a.sel_count[walk] = (int)min(n_open, (unsigned)a.max_sel);
+                if (n_open > (unsigned)a.max_sel) report(a.status, DEV_CAPACITY);
+            }
+            if (a.stats) {
+                zha_stats *st = a.stats + walk;
+                st->frontier[a.level] = (int)F;
+                st->opened[a.level] = (int)n_open;
+                if (a.level == 1) {
+                    long long sum = 0;
+                    for (int l = 1; l <= ZHA_MAX_DEPTH; ++l) sum += st->frontier[l];
+                    st->keys_read = (long long)a.C * n_open + a.tail;
+                    st->work = (long long)a.R * sum + st->keys_read;
+                }
+            }
+        }
+    }
+    chain_done();
+}
+
+template <int E>
+cudaError_t launch_select_warp(const SelectArgs &se, long long W, cudaStream_t st) {
+    SelectArgs a = se;
+    a.n_walks = W;
+    return launch_chained(select_warp_kernel<E>, dim3((unsigned)((W + 7) / 8)), dim3(256), 0, st, a);
+}
+
 template <int NT>
 cudaError_t launch_select(const SelectArgs &se, long long W, cudaStream_t st) {
     static bool smem_set = false;
@@ -1016,7 +1274,10 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
             if (mode == ZHA_TOP_K && l != start_level)
                 fmax = std::min<long long>(fmax, (long long)k * C + se.n_orph);
             Probe pr(t, ZHA_K_SELECT, st);
-            if (fmax > 8192 && W > 2LL * num_sms()) {
+            if (fmax <= 64) {
+                // frontiers of at most 64 nodes: one warp per walk
+                e = launch_select_warp<2>(se, W, st);
+            } else if (fmax > 8192 && W > 2LL * num_sms()) {
                 // many walks (prefill) over a wide level: most frontiers are far
                 // smaller than the level, so 256 threads and 4,096 keys of shared
                 // staging per CTA (wider frontiers stage in global memory) let more
