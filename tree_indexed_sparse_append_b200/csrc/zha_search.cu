@@ -36,9 +36,10 @@
 //                orphans of the level below form the next frontier (membership
 //                bits per walk and a per-tree union).
 //   select_warp_kernel  Levels whose frontiers hold at most 64 nodes (start
-//                levels of 64 nodes or fewer): one warp per walk, keys in
-//                registers, a bitonic sort across the warp, the same cutoff rule
-//                and the same fixed-point masses, so it opens the same nodes.
+//                levels of 64 nodes or fewer), or at most 512 in calls of many
+//                walks: one warp per walk, keys in registers, a bitonic sort
+//                across the warp, the same cutoff rule and the same fixed-point
+//                masses, so it opens the same nodes.
 #include <algorithm>
 #include <cmath>
 
@@ -151,6 +152,11 @@ __device__ __forceinline__ void red_or(unsigned *p, unsigned v) {
 }
 
 // Sets bits [lo, hi) of one walk's membership row and of its tree's union.
+// Trees of more than 8 walks (prefill) read the union word first: every walk of
+// the tree sets bits in the same words, and skipping the ones already set keeps
+// those reductions from queueing at a few L2 slices (bits are only ever set
+// during a search, so a stale read costs at most a redundant reduction). With
+// few walks the read would only add its latency.
 __device__ __forceinline__ void set_bits(unsigned *M_tree, unsigned *U_tree, int G, int g, long long lo,
                                          long long hi) {
     for (long long w = lo >> 5; w <= (hi - 1) >> 5; ++w) {
@@ -159,7 +165,7 @@ __device__ __forceinline__ void set_bits(unsigned *M_tree, unsigned *U_tree, int
         const int n = (int)(b1 - b0);
         const unsigned mask = (n == 32 ? FULL : ((1u << n) - 1u)) << (int)(b0 - (w << 5));
         red_or(&M_tree[w * G + g], mask);
-        red_or(&U_tree[w], mask);
+        if (G <= 8 || (__ldcg(&U_tree[w]) & mask) != mask) red_or(&U_tree[w], mask);
     }
 }
 
@@ -1277,6 +1283,13 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
             if (fmax <= 64) {
                 // frontiers of at most 64 nodes: one warp per walk
                 e = launch_select_warp<2>(se, W, st);
+            } else if (fmax <= 512 && W >= 8192) {
+                // many walks (prefill) over frontiers of at most 512 nodes: one
+                // warp per walk as well (with few walks the block path's shorter
+                // per-walk latency wins)
+                e = fmax <= 128   ? launch_select_warp<4>(se, W, st)
+                    : fmax <= 256 ? launch_select_warp<8>(se, W, st)
+                                  : launch_select_warp<16>(se, W, st);
             } else if (fmax > 8192 && W > 2LL * num_sms()) {
                 // many walks (prefill) over a wide level: most frontiers are far
                 // smaller than the level, so 256 threads and 4,096 keys of shared
