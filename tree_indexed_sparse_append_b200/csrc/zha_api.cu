@@ -180,7 +180,9 @@ int reserve(zha_tree *t, long long walks, int max_sel, Scratch *s) {
     if (c.d == 128 && Gw >= TC_MIN_G) {
         long long maxn_b = 0, maxn_sparse = 0;
         for (int l = 1; l <= t->max_depth; ++l) {
-            maxn_b = std::max(maxn_b, t->cap_nodes[l]);
+            // prepared B tiles serve the dense levels only (at most TC_MAX_NODES
+            // nodes scored); the sparse kernel splits its tiles itself
+            maxn_b = std::max(maxn_b, std::min(t->cap_nodes[l], TC_MAX_NODES));
             if (t->cap_nodes[l] > TC_MAX_NODES) maxn_sparse = std::max(maxn_sparse, t->cap_nodes[l]);
         }
         if (maxn_b > 0) tcl = tc_layout(t->T, Gw, maxn_b, maxn_sparse, c.R);

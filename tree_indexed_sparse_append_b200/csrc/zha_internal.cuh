@@ -280,8 +280,8 @@ cudaError_t launch_score_tc_queries(const zha_tree *t, const void *Q, int G, uns
 cudaError_t launch_score_tc(const zha_tree *t, int level, int G, unsigned char *atiles, unsigned char *btiles,
                             float *S, long long Sstride, cudaStream_t st);
 cudaError_t launch_score_tc_sparse(const zha_tree *t, int level, int G, const void *Q, const unsigned *M,
-                                   long long words, unsigned char *btiles, int *counts, int *lists, float *S,
-                                   long long Sstride, cudaStream_t st);
+                                   long long words, int *counts, int *lists, float *S, long long Sstride,
+                                   cudaStream_t st);
 // Records an error message for zha_last_error (this host thread); returns code.
 int set_error(int code, const char *msg);
 // Grows the tree's second scratch block (full-scan indexer, chunk-mass profile,

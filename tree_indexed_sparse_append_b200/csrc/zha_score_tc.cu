@@ -35,11 +35,14 @@
 //   cover a small part of them):
 //   tc_members       per tree and tile of 16 nodes (one word of the membership
 //                    bitmap), the list of walks whose frontier holds one of them.
-//   score_tc_sparse_kernel  one CTA per tile with members: the tile's three key
-//                    parts and biases in shared memory (one bulk copy), the member
-//                    walks' queries gathered 128 at a time (cp.async, zero-filled
-//                    past the end), the same MMAs into 128 TMEM columns, and scores
-//                    stored for the member walks only.
+//   score_tc_sparse_kernel  persistent, one CTA per SM over the tiles with
+//                    members: the tile's fp32 node rows in one bulk copy (issued
+//                    while the previous tile is multiplied), split into the three
+//                    parts in shared memory; the member walks' queries gathered 128
+//                    at a time (cp.async, zero-filled past the end) into two
+//                    alternating buffers; the same MMAs into two alternating TMEM
+//                    accumulators, so a batch's MMAs overlap the previous batch's
+//                    epilogue; scores stored for the member walks only.
 // Every wait is bounded: on timeout the kernel records DEV_TIMEOUT, waits (also
 // bounded) for its own copies and MMAs, frees its TMEM and returns.
 #include <cstdint>
@@ -413,7 +416,9 @@ __global__ void __launch_bounds__(256) tc_members_kernel(MembersArgs a) {
 }
 
 struct SparseArgs {
-    const unsigned char *btiles;  // [T][ntiles][TC_BTILE]
+    const float *nodes;           // the level's nodes [T][cap][NF] (fp32 keys [R][D], then biases)
+    long long node_tree;          // floats per tree
+    int NF, R, T;
     const __nv_bfloat16 *Q;       // [T * G][128]
     const int *counts, *lists;
     long long ntiles, n_level;
@@ -425,37 +430,63 @@ struct SparseArgs {
     unsigned long long wait_ns;  // limit of every wait
 };
 
-constexpr int TS_SMEM = 3 * TC_PART + TC_ATILE + TC_N * 4 + 64;  // B tile, gathered walks, biases, barriers
+// Shared memory of the sparse kernel: a tile's fp32 node rows (one bulk copy),
+// two buffers of gathered queries, the three bf16 key parts, the biases, barriers
+// (230,976 bytes in all).
+constexpr int TS_X = TC_N * (TC_K + 1) * 4;  // 128 columns of 128 keys and a bias, at most
+constexpr int TS_A_OFF = (TS_X + 1023) & ~1023;
+constexpr int TS_P_OFF = TS_A_OFF + 2 * TC_ATILE;
+constexpr int TS_BIAS_OFF = TS_P_OFF + 3 * TC_PART;
+constexpr int TS_BAR_OFF = TS_BIAS_OFF + TC_N * 4;
+constexpr int TS_SMEM = TS_BAR_OFF + 64;
 
-
+// Persistent: one CTA per SM takes the B tiles with members (NPT consecutive
+// nodes x RP references = 128 columns) in turn. A tile's fp32 rows arrive in one
+// bulk copy, issued while the previous tile is still being multiplied, and are
+// split into the hi, mid and lo parts in shared memory (no preparation pass, 4
+// bytes read per key element). The member walks' queries are gathered 128 at a
+// time into two alternating buffers (the first batch's while the rows arrive),
+// and the MMAs of a batch write one of two TMEM accumulators: while the epilogue
+// reads batch b, the MMAs of batch b + 1 run and the queries of batch b + 2 are
+// gathered.
 template <int RP>
 __global__ void __launch_bounds__(128, 1) score_tc_sparse_kernel(SparseArgs a) {
     constexpr int NPT = TC_N / RP;
     extern __shared__ __align__(16) unsigned char smem[];  // no static shared memory: all of it is here
-    unsigned char *sB = smem;                              // the tile's three key parts
-    unsigned char *sA = smem + 3 * TC_PART;                // 128 gathered queries
-    float *sBias = reinterpret_cast<float *>(smem + 3 * TC_PART + TC_ATILE);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 3 * TC_PART + TC_ATILE + TC_N * 4);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2);
+    unsigned char *sX = smem;                               // node rows of the next tile to split
+    unsigned char *sA = smem + TS_A_OFF;                    // query buffers 0 and 1
+    unsigned char *sP = smem + TS_P_OFF;                    // the tile's three key parts
+    float *sBias = reinterpret_cast<float *>(smem + TS_BIAS_OFF);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TS_BAR_OFF);  // rows copy, MMAs of buffer 0, of buffer 1
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3);
+    volatile int *s_ok = reinterpret_cast<volatile int *>(bars + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const long long nt = blockIdx.x, t = blockIdx.y;
-    const long long tn = t * a.ntiles + nt;
-    const int count = a.counts[tn];
-    if (count <= 0) return;  // the same for the whole CTA; nothing allocated yet
-    const int *list = a.lists + tn * a.G;
-    const uint32_t barB = smem_u32(bars), barM = smem_u32(bars + 1);
+    const long long n_tiles = (long long)a.T * a.ntiles;
+    // the next tile with members from `from` on, in this CTA's stride (-1: none)
+    auto next_tile = [&](long long from) -> long long {
+        for (long long i = from; i < n_tiles; i += gridDim.x)
+            if (a.counts[i] > 0) return i;
+        return -1;
+    };
+    long long cur = next_tile(blockIdx.x);
+    if (cur < 0) return;  // the same for the whole CTA; nothing allocated yet
+
+    const uint32_t barX = smem_u32(bars);
+    const uint32_t barM0 = smem_u32(bars + 1), barM1 = smem_u32(bars + 2);
+    auto barM = [&](int buf) { return buf ? barM1 : barM0; };
     const unsigned long long lim = a.wait_ns;
     auto mbar_wait = [lim](uint32_t bar, uint32_t phase) { return zha::mbar_wait(bar, phase, lim); };
 
     if (tid == 0) {
-        mbar_init(barB, 1);
-        mbar_init(barM, 1);
+        mbar_init(barX, 1);
+        mbar_init(barM0, 1);
+        mbar_init(barM1, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(TC_N)
+                     "r"(2 * TC_N)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -463,89 +494,181 @@ __global__ void __launch_bounds__(128, 1) score_tc_sparse_kernel(SparseArgs a) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    if (tid == 0) {
-        const unsigned char *src = a.btiles + tn * TC_BTILE;
-        mbar_expect_tx(barB, 3 * TC_PART + TC_N * 4);
-        bulk_g2s(smem_u32(sB), src, 3 * TC_PART, barB);
-        bulk_g2s(smem_u32(sBias), src + 3 * TC_PART, TC_N * 4, barB);
-    }
-    bool ok = mbar_wait(barB, 0);
-    bool b_done = ok, m_pending = false;
-    uint32_t phase = 0;
-    for (int c0 = 0; c0 < count; c0 += TC_M) {
-        if (!__syncthreads_and(ok)) {
-            ok = false;
-            break;
-        }
+
+    auto tile_nodes = [&](long long tile) {  // nodes of the tile that exist
+        const long long n0 = (tile % a.ntiles) * NPT;
+        return (int)(a.n_level - n0 < NPT ? a.n_level - n0 : NPT);
+    };
+    auto copy_rows = [&](long long tile) {  // one thread
+        const long long tt = tile / a.ntiles, n0 = (tile % a.ntiles) * NPT;
+        const uint32_t bytes = (uint32_t)tile_nodes(tile) * (uint32_t)a.NF * 4u;  // NF * 4 is a multiple of 16
+        mbar_expect_tx(barX, bytes);
+        bulk_g2s(smem_u32(sX), a.nodes + tt * a.node_tree + n0 * a.NF, bytes, barX);
+    };
+    // thread i brings walk list[b * 128 + i]'s query into buffer buf (zeros past
+    // the list); returns the walk (-1 past the list)
+    auto gather = [&](long long tt, const int *list, int count, int b, int buf) -> int {
+        const int c0 = b * TC_M;
         const int rows = min(TC_M, count - c0);
-        // gather: thread i brings walk list[c0 + i]'s query (zeros past the list)
         const int g = tid < rows ? list[c0 + tid] : -1;
-        const __nv_bfloat16 *src = a.Q + ((long long)t * a.G + (g >= 0 ? g : 0)) * TC_K;
-        const uint32_t dst = smem_u32(sA);
+        const __nv_bfloat16 *src = a.Q + (tt * a.G + (g >= 0 ? g : 0)) * TC_K;
+        const uint32_t dst = smem_u32(sA + buf * TC_ATILE);
 #pragma unroll
         for (int kc = 0; kc < TC_K / 8; ++kc) cp_async16(dst + core_offset(tid, kc * 8), src + kc * 8, g >= 0 ? 16u : 0u);
         asm volatile("cp.async.commit_group;" ::: "memory");
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic-proxy writes -> MMA reads
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
-#pragma unroll
-            for (int part = 0; part < 3; ++part)
-#pragma unroll
-                for (int ks = 0; ks < TC_K / 16; ++ks)
-                    tc_mma(tmem, smem_desc(a0 + ks * 256), smem_desc(b0 + part * TC_PART + ks * 256),
-                           (part | ks) ? 1u : 0u);
-            tc_commit(barM);
-        }
-        // one thread waits for the MMAs and tells the others, so that every warp
-        // takes the same branch before the warp-collective TMEM loads
-        volatile int *s_ok = reinterpret_cast<volatile int *>(bars + 3);
-        if (tid == 0) *s_ok = mbar_wait(barM, phase) ? 1 : 0;
-        __syncthreads();
-        if (!*s_ok) {
-            ok = false;
-            m_pending = true;
-            break;
-        }
-        phase ^= 1u;
+        return g;
+    };
+    auto issue = [&](int buf) {  // one thread: the batch in buffer buf against the three parts
         tc_fence_after();
-        float sc[TC_N];
+        const uint32_t a0 = smem_u32(sA + buf * TC_ATILE), b0 = smem_u32(sP);
 #pragma unroll
-        for (int cc = 0; cc < TC_N; cc += 16) {
-            float v[16];
-            tc_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)cc, v);
+        for (int part = 0; part < 3; ++part)
 #pragma unroll
-            for (int i = 0; i < 16; ++i) sc[cc + i] = v[i];
+            for (int ks = 0; ks < TC_K / 16; ++ks)
+                tc_mma(tmem + buf * TC_N, smem_desc(a0 + ks * 256), smem_desc(b0 + part * TC_PART + ks * 256),
+                       (part | ks) ? 1u : 0u);
+        tc_commit(barM(buf));
+    };
+
+    // waits outstanding, and the phase of each barrier
+    bool pendX = false, pend0 = false, pend1 = false;
+    uint32_t phX = 0u, ph0 = 0u, ph1 = 0u;
+    if (tid == 0) copy_rows(cur);
+    pendX = true;
+    bool ok = true;
+    while (ok && cur >= 0) {
+        const long long tt = cur / a.ntiles;
+        const long long n0 = (cur % a.ntiles) * NPT;
+        const int nv = tile_nodes(cur);
+        const int count = a.counts[cur];
+        const int *list = a.lists + cur * a.G;
+        const int nb = (count + TC_M - 1) / TC_M;
+        // the first batch's queries while the rows arrive (every MMA of the
+        // previous tile is complete, so both buffers are free)
+        int g_cur = gather(tt, list, count, 0, 0);
+        ok = __syncthreads_and(mbar_wait(barX, phX));
+        if (!ok) break;
+        pendX = false;
+        phX ^= 1u;
+        {
+            // split: item -> column c (8 consecutive columns per 8 threads, so a
+            // quarter warp's 16-byte part stores are contiguous) and 8-key chunk kc,
+            // rotated by the column so that the row reads spread over the banks
+            const float *X = reinterpret_cast<const float *>(sX);
+            for (int item = tid; item < TC_N * (TC_K / 8); item += 128) {
+                const int c = ((item >> 7) << 3) | (item & 7);
+                const int kc = (((item >> 3) & 15) + (item & 7)) & 15;
+                const int q = c / RP, r = c % RP;
+                uint32_t hw[4] = {0u, 0u, 0u, 0u}, mw[4] = {0u, 0u, 0u, 0u}, lw[4] = {0u, 0u, 0u, 0u};
+                if (q < nv && r < a.R) {
+                    const float *src = X + (long long)q * a.NF + r * TC_K + kc * 8;
+                    const float4 x0 = *reinterpret_cast<const float4 *>(src);
+                    const float4 x1 = *reinterpret_cast<const float4 *>(src + 4);
+                    const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            const float v = x[2 * i + jj];
+                            const __nv_bfloat16 h = __float2bfloat16_rn(v);
+                            const float r1 = v - __bfloat162float(h);
+                            const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+                            const __nv_bfloat16 l = __float2bfloat16_rn(r1 - __bfloat162float(m));
+                            hw[i] |= (uint32_t)__bfloat16_as_ushort(h) << (16 * jj);
+                            mw[i] |= (uint32_t)__bfloat16_as_ushort(m) << (16 * jj);
+                            lw[i] |= (uint32_t)__bfloat16_as_ushort(l) << (16 * jj);
+                        }
+                    }
+                }
+                const int off = core_offset(c, kc * 8);
+                *reinterpret_cast<uint4 *>(sP + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(sP + TC_PART + off) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+                *reinterpret_cast<uint4 *>(sP + 2 * TC_PART + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+            const int c = tid, q = c / RP, r = c % RP;  // 128 threads, 128 columns
+            sBias[c] = (q < nv && r < a.R) ? X[(long long)q * a.NF + (long long)a.R * TC_K + r] : -INFINITY;
         }
-        tc_wait_ld();
-        tc_fence_before();
-#pragma unroll
-        for (int q = 0; q < NPT; ++q) {
-            float mx = -INFINITY;
-#pragma unroll
-            for (int r = 0; r < RP; ++r) mx = fmaxf(mx, fmaf(a.beta, sc[q * RP + r], sBias[q * RP + r]));
-            sc[q] = mx;
+        // the parts (generic-proxy writes) are read by the MMAs; every row is read
+        // before the next tile's copy overwrites them
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+        const long long nxt = next_tile(cur + gridDim.x);
+        if (nxt >= 0) {
+            if (tid == 0) copy_rows(nxt);
+            pendX = true;
         }
-        if (g >= 0) {
-            float *Srow = a.S + ((long long)t * a.G + g) * a.Sstride + nt * NPT;
+        if (tid == 0) issue(0);
+        pend0 = true;
+        for (int b = 0; b < nb; ++b) {
+            const int buf = b & 1;
+            int g_next = -1;
+            if (b + 1 < nb) g_next = gather(tt, list, count, b + 1, buf ^ 1);  // batch b - 1's MMAs are complete
+            // one thread waits for batch b's MMAs and tells the others, so that every
+            // warp takes the same branch before the warp-collective TMEM loads
+            if (tid == 0) *s_ok = mbar_wait(barM(buf), buf ? ph1 : ph0) ? 1 : 0;
+            __syncthreads();
+            if (!*s_ok) {
+                ok = false;
+                break;
+            }
+            if (buf) {
+                pend1 = false;
+                ph1 ^= 1u;
+            } else {
+                pend0 = false;
+                ph0 ^= 1u;
+            }
+            if (b + 1 < nb) {
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncthreads();  // also: batch b - 1's TMEM reads (buffer buf ^ 1) are done
+                if (tid == 0) issue(buf ^ 1);
+                if (buf) pend0 = true;
+                else pend1 = true;
+            }
+            tc_fence_after();
+            float sc[TC_N];
 #pragma unroll
-            for (int q = 0; q < NPT; ++q)
-                if (nt * NPT + q < a.n_level) Srow[q] = sc[q];
+            for (int cc = 0; cc < TC_N; cc += 16) {
+                float v[16];
+                tc_ld16(tmem + buf * TC_N + ((uint32_t)(warp * 32) << 16) + (uint32_t)cc, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sc[cc + i] = v[i];
+            }
+            tc_wait_ld();
+            tc_fence_before();
+#pragma unroll
+            for (int q = 0; q < NPT; ++q) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int r = 0; r < RP; ++r) mx = fmaxf(mx, fmaf(a.beta, sc[q * RP + r], sBias[q * RP + r]));
+                sc[q] = mx;
+            }
+            if (g_cur >= 0) {
+                float *Srow = a.S + (tt * a.G + g_cur) * a.Sstride + n0;
+#pragma unroll
+                for (int q = 0; q < NPT; ++q)
+                    if (q < nv) Srow[q] = sc[q];
+            }
+            g_cur = g_next;
         }
+        __syncthreads();  // every TMEM read and bias read of this tile is done
+        cur = nxt;
     }
-    if (!ok) {
-        if (tid == 0) report(a.status, DEV_TIMEOUT);
-        // copies and MMAs still in flight finish before the memory goes away
-        if (!b_done) (void)mbar_wait(barB, 0);
-        if (m_pending) (void)mbar_wait(barM, phase);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");  // no gather lands after the CTA
+    if (!ok && tid == 0) {
+        report(a.status, DEV_TIMEOUT);
+        // the copy and MMAs still in flight finish before the memory goes away
+        if (pendX) (void)mbar_wait(barX, phX);
+        if (pend0) (void)mbar_wait(barM0, ph0);
+        if (pend1) (void)mbar_wait(barM1, ph1);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_N) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * TC_N) : "memory");
 }
 
 template <int RP>
@@ -558,22 +681,23 @@ cudaError_t launch_sparse_rp(const zha_tree *t, const SparseArgs &sa, cudaStream
         attr = true;
     }
     Probe pr(t, ZHA_K_SCORE_TC, st);
-    score_tc_sparse_kernel<RP><<<dim3((unsigned)sa.ntiles, (unsigned)t->T), 128, TS_SMEM, st>>>(sa);
+    long long grid = sa.ntiles * t->T;  // persistent: one CTA per SM at most
+    if (grid > num_sms()) grid = num_sms();
+    score_tc_sparse_kernel<RP><<<(unsigned)grid, 128, TS_SMEM, st>>>(sa);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_score_tc_sparse(const zha_tree *t, int level, int G, const void *Q, const unsigned *M,
-                                   long long words, unsigned char *btiles, int *counts, int *lists, float *S,
-                                   long long Sstride, cudaStream_t st) {
+                                   long long words, int *counts, int *lists, float *S, long long Sstride,
+                                   cudaStream_t st) {
     const zha_config &c = t->cfg;
     int RP = 1;
     while (RP < c.R) RP <<= 1;
     const long long n_level = t->n_nodes[level];
     const long long ntiles = (n_level * RP + TC_N - 1) / TC_N;
-    cudaError_t e = launch_prep_keys(t, level, RP, ntiles, btiles, st);
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
     MembersArgs m{};
     m.M = M;
     m.words = words;
@@ -588,7 +712,11 @@ cudaError_t launch_score_tc_sparse(const zha_tree *t, int level, int G, const vo
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     SparseArgs sa{};
-    sa.btiles = btiles;
+    sa.nodes = t->nodes[level];
+    sa.node_tree = t->cap_nodes[level] * t->NF;
+    sa.NF = t->NF;
+    sa.R = c.R;
+    sa.T = t->T;
     sa.Q = static_cast<const __nv_bfloat16 *>(Q);
     sa.counts = counts;
     sa.lists = lists;

@@ -1235,7 +1235,7 @@ cudaError_t launch_search(const zha_tree *t, const Scratch &s, const void *Q, zh
             e = launch_score_tc(t, l, G, s.tc, s.tc_b, s.S, s.Sstride, st);
             if (e != cudaSuccess) return e;
         } else if (s.tc_lists && tc_sparse_applicable(t, G, Q, q_dtype, l)) {
-            e = launch_score_tc_sparse(t, l, G, Q, s.M[l], words(l), s.tc_b, s.tc_counts, s.tc_lists, s.S, s.Sstride,
+            e = launch_score_tc_sparse(t, l, G, Q, s.M[l], words(l), s.tc_counts, s.tc_lists, s.S, s.Sstride,
                                        st);
             if (e != cudaSuccess) return e;
         } else {
