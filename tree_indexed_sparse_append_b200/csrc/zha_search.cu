@@ -501,7 +501,12 @@ __device__ __forceinline__ int fine_bucket(float s, float m, int cb) {
     return y >= 255.f ? 255 : (y > 0.f ? (int)y : 0);
 }
 
-template <int NT>
+// KB: keys loaded together per thread in the passes over the frontier: 8 for the
+// full scan, whose frontier (every key of the tree) is staged in global memory,
+// so that a pass does not wait one round trip per position; 1 for the tree
+// walk, whose frontiers sit in shared memory, which keeps the registers for the
+// rest (batched loads made those selections slower).
+template <int NT, int KB>
 __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
     chain_start();
     extern __shared__ uint32_t skey_s[];
@@ -583,14 +588,22 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
             if (tid == 0) s_ncand = 0;
             __syncthreads();
             const int shift = 24 - 8 * (stage - 2);
-            for (long long i = tid; i < F; i += NT) {
-                const uint32_t k = key_at(i);
+            // keys in batches of KB strided positions, loaded before any is used
+            for (long long i0 = tid; i0 < F; i0 += KB * NT) {
+              uint32_t kk[KB];
+#pragma unroll
+              for (int u = 0; u < KB; ++u) kk[u] = i0 + u * NT < F ? key_at(i0 + u * NT) : 0u;
+#pragma unroll
+              for (int u = 0; u < KB; ++u) {
+                if (i0 + u * NT >= F) break;
+                const uint32_t k = kk[u];
                 if (!in_play(k, stage)) continue;
                 const float s = key_to_float(k);
                 const int b = stage == 0 ? coarse_bucket(s, m)
                                          : (stage == 1 ? fine_bucket(s, m, cb) : (int)((k >> shift) & 255));
                 atomicAdd(&h_cnt[wcopy][b], 1u);
                 if (top_p) add_mass(&h_mlo[wcopy][b], &h_mhi[wcopy][b], mass(s));
+              }
             }
             __syncthreads();
             // threads 0..255 own one bucket each: buckets ascend from the highest
@@ -639,11 +652,16 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
             }
             if (cnt <= CAND_MAX) {
                 // few keys left: list them and let one warp rank them directly
-                for (long long i = tid; i < F; i += NT) {
-                    const uint32_t k = key_at(i);
-                    if (in_play(k, stage + 1)) {
-                        const unsigned slot = atomicAdd(&s_ncand, 1u);
-                        if (slot < CAND_MAX) s_cand[slot] = k;
+                for (long long i0 = tid; i0 < F; i0 += KB * NT) {
+                    uint32_t kk[KB];
+#pragma unroll
+                    for (int u = 0; u < KB; ++u) kk[u] = i0 + u * NT < F ? key_at(i0 + u * NT) : 0u;
+#pragma unroll
+                    for (int u = 0; u < KB; ++u) {
+                        if (i0 + u * NT < F && in_play(kk[u], stage + 1)) {
+                            const unsigned slot = atomicAdd(&s_ncand, 1u);
+                            if (slot < CAND_MAX) s_cand[slot] = kk[u];
+                        }
                     }
                 }
                 __syncthreads();
@@ -729,13 +747,13 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
         eq_base = __shfl_sync(FULL, eq_base, 0);
     }
     // is position i opened? `eq` is the number of keys equal to kstar before this group
-    auto opened = [&](long long i, unsigned eq, unsigned &eq_in_group) -> bool {
+    // (key: the key at i, loaded by the caller)
+    auto opened = [&](long long i, uint32_t key, unsigned eq, unsigned &eq_in_group) -> bool {
         const bool in = i < rend;
         if (open_all) {
             eq_in_group = 0;
             return in;
         }
-        const uint32_t key = in ? key_at(i) : 0u;
         const bool is_eq = in && key == kstar;
         const unsigned eqm = __ballot_sync(FULL, is_eq);
         eq_in_group = __popc(eqm);
@@ -744,10 +762,22 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
     unsigned open_w = 0;
     {
         unsigned eq = eq_base, eqg;
-        for (long long i0 = rbeg; i0 < rend; i0 += 32) {
-            const bool o = opened(i0 + lane, eq, eqg);
-            open_w += __popc(__ballot_sync(FULL, o));
-            eq += eqg;
+        // keys of KB groups of 32 positions are loaded before any is used
+        for (long long i00 = rbeg; i00 < rend; i00 += 32 * KB) {
+            uint32_t kk[KB];
+#pragma unroll
+            for (int u = 0; u < KB; ++u) {
+                const long long i = i00 + 32 * u + lane;
+                kk[u] = i < rend && !open_all ? key_at(i) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < KB; ++u) {
+                const long long i0 = i00 + 32 * u;
+                if (i0 >= rend) break;
+                const bool o = opened(i0 + lane, kk[u], eq, eqg);
+                open_w += __popc(__ballot_sync(FULL, o));
+                eq += eqg;
+            }
         }
     }
     unsigned n_open;
@@ -763,17 +793,22 @@ __global__ void __launch_bounds__(NT) select_level_kernel(SelectArgs a) {
         // node ids of 8 groups of 32 positions are loaded before any is used
         for (long long i00 = rbeg; i00 < rend; i00 += 32 * 8) {
             long long idv[8];
+            uint32_t kk[KB > 1 ? 8 : 1];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const long long i = i00 + 32 * u + lane;
                 idv[u] = i < rend ? frontier_id(a, lid, par, npar, i) : 0;
+                if constexpr (KB > 1) kk[u] = i < rend && !open_all ? key_at(i) : 0u;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const long long i0 = i00 + 32 * u;
                 if (i0 >= rend) break;
                 const long long i = i0 + lane;
-                const bool o = opened(i, eq, eqg);
+                uint32_t key;
+                if constexpr (KB > 1) key = kk[u];
+                else key = i < rend && !open_all ? key_at(i) : 0u;
+                const bool o = opened(i, key, eq, eqg);
                 const unsigned om = __ballot_sync(FULL, o);
                 if (o) {
                     const unsigned r = rank + __popc(om & below);
@@ -1067,17 +1102,17 @@ cudaError_t launch_select_warp(const SelectArgs &se, long long W, cudaStream_t s
     return launch_chained(select_warp_kernel<E>, dim3((unsigned)((W + 7) / 8)), dim3(256), 0, st, a);
 }
 
-template <int NT>
+template <int NT, int KB = 1>
 cudaError_t launch_select(const SelectArgs &se, long long W, cudaStream_t st) {
     static bool smem_set = false;
     if (!smem_set) {
-        cudaError_t e = cudaFuncSetAttribute(select_level_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             16384 * (int)sizeof(uint32_t));
+        cudaError_t e = cudaFuncSetAttribute(select_level_kernel<NT, KB>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 16384 * (int)sizeof(uint32_t));
         if (e != cudaSuccess) return e;
         smem_set = true;
     }
-    return launch_chained(select_level_kernel<NT>, dim3((unsigned)W), dim3(NT), (size_t)se.smem_keys * sizeof(uint32_t),
-                          st, se);
+    return launch_chained(select_level_kernel<NT, KB>, dim3((unsigned)W), dim3(NT),
+                          (size_t)se.smem_keys * sizeof(uint32_t), st, se);
 }
 
 template <int D, int RP>
@@ -1155,7 +1190,7 @@ cudaError_t launch_select_all(const zha_tree *t, const float *S, uint32_t *gkey,
     Probe pr(t, ZHA_K_SELECT, st);
     if (N > 8192) {
         se.smem_keys = std::min<long long>(N, 16384);
-        return launch_select<1024>(se, W, st);
+        return N > 16384 ? launch_select<1024, 8>(se, W, st) : launch_select<1024>(se, W, st);
     }
     se.smem_keys = N;
     return launch_select<256>(se, W, st);
