@@ -314,6 +314,18 @@ def test_large_frontiers():
                                  (O.TOP_K, 0, 1500)))
 
 
+@pytest.mark.parametrize("N", [8192, 16384])
+def test_many_walks_warp_selector(N):
+    # 8,192 walks (a prefill-sized call) on trees of C = 4, depth 6: 8,192 keys give
+    # levels of 2,048, 512, 128, 32, 8 and 2 nodes, 16,384 keys levels of 4,096,
+    # 1,024, 256, 64, 16 and 4, so the walk starts at 32 or 64 nodes and the levels
+    # of 128, 256 and 512 nodes are selected by the one-warp-per-walk selector with
+    # 4, 8 and 16 keys per lane; every walk is checked against the oracle
+    K, V, refs, Q = _tiny(N, C=4, depth=6, d=64, R=4, nq=8192, seed=11)
+    _check_against_oracle(K, V, refs, Q, N, 4, 6, 0.125, top_width=64,
+                          modes=((O.TOP_P, 0.9, 0), (O.TOP_K, 0, 3)))
+
+
 def test_max_sel_overflow_is_reported():
     Z = zha()
     K, V, refs, Q = _tiny(1024, C=8, depth=2)
